@@ -1,0 +1,76 @@
+"""Workload table for the block-sparse global attention layer.
+
+Each workload is one global-attention layer of a VGGT-style multi-view geometry
+transformer: F frames, each with P patch tokens and S special tokens (1 camera +
+4 register), H heads of width d, and the block-selection hyper-parameters b
+(block size), rho (sparsity floor) and tau (CDF coverage) named in
+"Block-Sparse Global Attention for Efficient Multi-View Geometry Transformers",
+section 损失函数 / 训练策略 (the only tunables are tau, rho and b).
+
+Shapes follow that page's workloads: 518x518 input -> 37x37 = 1369 patches per
+frame; 294x518 input -> 21x37 = 777 patches per frame.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, replace
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    frames: int            # F
+    patch_per_frame: int   # P
+    special_per_frame: int  # S (prefix of each frame)
+    heads: int             # H
+    head_dim: int          # d
+    block: int             # b
+    rho: float             # sparsity floor: k = floor(B (1 - rho))
+    tau: float             # CDF coverage threshold
+    dtype: str             # "f32" or "bf16"
+    planting: str          # "tiny" (permuted cross-frame copies) or "five_percent"
+    head_budgets: bool = False  # per-head densities from capped water-filling
+    seed: int = 0
+
+    @property
+    def tokens_per_frame(self) -> int:
+        return self.patch_per_frame + self.special_per_frame
+
+    @property
+    def n_tokens(self) -> int:
+        return self.frames * self.tokens_per_frame
+
+    @property
+    def n_patch(self) -> int:
+        return self.frames * self.patch_per_frame
+
+    @property
+    def n_special(self) -> int:
+        return self.frames * self.special_per_frame
+
+    @property
+    def n_blocks(self) -> int:
+        return -(-self.n_patch // self.block)
+
+    def with_(self, **kw) -> "Workload":
+        return replace(self, **kw)
+
+
+TINY = Workload("tiny", 2, 64, 5, 2, 64, 16, 0.5, 0.9, "f32", "tiny")
+VGGT518 = Workload("vggt518", 10, 1369, 5, 16, 64, 64, 0.5, 0.9, "bf16", "five_percent")
+SWEEP_R50 = Workload("sweep_r50", 32, 777, 5, 16, 64, 64, 0.5, 0.95, "bf16", "five_percent")
+SWEEP_R75 = SWEEP_R50.with_(name="sweep_r75", rho=0.75)
+SWEEP_R90 = SWEEP_R50.with_(name="sweep_r90", rho=0.9)
+# tau is not given for the per-head-budget workload; tau = 0 makes each head keep
+# exactly its budgeted k_h blocks so that the layer density is the budget (1 - rho).
+PERHEAD100 = Workload("perhead100", 100, 777, 5, 16, 64, 128, 0.75, 0.0, "bf16",
+                      "five_percent", head_budgets=True)
+PERHEAD100_TAU95 = PERHEAD100.with_(name="perhead100_tau95", tau=0.95)
+LONG500 = Workload("long500", 500, 777, 5, 16, 64, 128, 0.9, 0.95, "bf16", "five_percent")
+
+# Non-degenerate variants: with the near-uniform pooled distributions of this
+# generator, tau >= 0.9 keeps almost every block; tau = 0 exercises the top-k floor.
+TINY_TAU0 = TINY.with_(name="tiny_tau0", tau=0.0)
+SWEEP_TAU0 = SWEEP_R75.with_(name="sweep_tau0", tau=0.0)
+
+ALL = {w.name: w for w in (TINY, VGGT518, SWEEP_R50, SWEEP_R75, SWEEP_R90, PERHEAD100,
+                           PERHEAD100_TAU95, LONG500, TINY_TAU0, SWEEP_TAU0)}
