@@ -1,0 +1,377 @@
+"""Benchmark of the block-sparse global-attention layer on B200.
+
+One step = one whole layer on one GPU: pool -> mask -> pack -> special dense ->
+block-sparse attention -> merge, on seeded synthetic inputs already resident in HBM.
+Default workload: 100 frames x (777 patch + 5 special) tokens, 16 heads, d = 64, b = 128,
+layer budget rho = 0.75 split across heads by capped water-filling of LogNormal(0, 1)
+scores, tau = 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Prints one JSON line (rank 0). With N > 1 (torchrun), every rank runs its own replica of
+the layer (the layer has no exchange step); time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from view_transformers_b200 import configs, synth  # noqa: E402
+
+METRIC = "global-attn ms/layer & effective TFLOPS vs dense at 100 frames, rho=0.75"
+UNIT = "ms/layer"
+STAGES = ["pool", "mask", "pack", "special", "sparse", "merge"]
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p["hbm_gbs"], p["bf16_tflops"], p["bf16_tflops_sustained"], "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            self.proc.wait(timeout=10)
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        try:
+            for line in open(self.path):
+                f = [x.strip() for x in line.split(",")]
+                if len(f) < 9:
+                    continue
+                try:
+                    sm.append(float(f[1]))
+                    mx.append(float(f[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, f[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        finally:
+            os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------- helpers
+def sparse_flops(kv_cnt, kv_idx, w) -> float:
+    """4 d sum_h sum_(i, j kept) |I_i| |J_j| over patch query/key blocks."""
+    B, b, Np = w.n_blocks, w.block, w.n_patch
+    sizes = np.minimum(b, Np - np.arange(B) * b).astype(np.float64)       # |I_j|
+    valid = np.arange(B)[None, None, :] < kv_cnt[:, :, None]
+    keys = np.where(valid, sizes[np.minimum(kv_idx.astype(np.int64), B - 1)], 0.0).sum(axis=2)   # [H, B]
+    return float(4 * w.head_dim * (keys * sizes[None, :]).sum())
+
+
+def special_flops(w) -> float:
+    return float(4 * w.head_dim * w.heads * (w.n_special * w.n_tokens + w.n_patch * w.n_special))
+
+
+def stage_bytes(w) -> dict:
+    e = 2 if w.dtype == "bf16" else 4
+    row = w.heads * w.head_dim
+    B = w.n_blocks
+    pooled = 2 * w.heads * B * w.head_dim * 4
+    return {
+        "pool": 2 * w.n_patch * row * e + pooled,
+        "pack": 3 * w.n_tokens * row * e + 3 * w.n_tokens * row * 2,
+        "merge": 2 * w.n_patch * row * 4 + 2 * w.heads * w.n_patch * 4 + w.n_patch * row * e,
+    }
+
+
+def run_steps(torch, L, q, k, v, steps, record_stages=True):
+    """Runs `steps` layers; returns per-step stage durations (ms) and the total (ms)."""
+    st = torch.cuda.current_stream()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)] for _ in range(steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    b = L.buf
+    from view_transformers_b200 import _lib
+    sp = st.cuda_stream
+    status = b.status.data_ptr()
+    start.record(st)
+    for s in range(steps):
+        e = evs[s]
+        e[0].record(st)
+        _lib.bsa_pool_qk(L.layout, q.data_ptr(), k.data_ptr(), b.pq.data_ptr(), b.pk.data_ptr(), status, sp)
+        e[1].record(st)
+        _lib.bsa_predict_mask(L.layout, b.pq.data_ptr(), b.pk.data_ptr(), L.rho, L.tau, L.head_density,
+                              b.mask_bits.data_ptr(), b.kv_idx.data_ptr(), b.kv_cnt.data_ptr(), status, sp)
+        e[2].record(st)
+        _lib.bsa_pack_qkv(L.layout, q.data_ptr(), k.data_ptr(), v.data_ptr(), L.ws_ptr, L.ws_bytes, status, sp)
+        e[3].record(st)
+        _lib.bsa_special_dense(L.layout, q.data_ptr(), k.data_ptr(), v.data_ptr(), L.ws_ptr, L.ws_bytes,
+                               b.out.data_ptr(), b.o_ps.data_ptr(), b.lse_ps.data_ptr(), status, sp)
+        e[4].record(st)
+        _lib.bsa_block_sparse_attn(L.layout, q.data_ptr(), k.data_ptr(), v.data_ptr(), L.ws_ptr, L.ws_bytes,
+                                   b.kv_idx.data_ptr(), b.kv_cnt.data_ptr(), b.o_pp.data_ptr(),
+                                   b.lse_pp.data_ptr(), status, sp)
+        e[5].record(st)
+        _lib.bsa_merge(L.layout, b.o_pp.data_ptr(), b.lse_pp.data_ptr(), b.o_ps.data_ptr(), b.lse_ps.data_ptr(),
+                       b.out.data_ptr(), status, sp)
+        e[6].record(st)
+    end.record(st)
+    end.synchronize()
+    per_stage = {name: [evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(steps)]
+                 for i, name in enumerate(STAGES)}
+    return per_stage, start.elapsed_time(end)
+
+
+LAUNCHES_PER_STEP = {"pool": 1, "mask": 1, "pack": 1, "special": 2, "sparse": 1, "merge": 1}
+
+
+# ---------------------------------------------------------------------------- CPU oracle
+def oracle_layer_sample(w, x, budget_s: float, seed: int = 7):
+    """Times the fp64 oracle on a bounded sample of one layer and scales it to ms/layer.
+
+    Full pooling and mask prediction; attention for a seeded sample of (head, query block)
+    pairs plus a seeded sample of special query rows, scaled by the sampled fraction."""
+    import oracle
+    from threadpoolctl import threadpool_info
+    lay = oracle.Layout(w.frames, w.tokens_per_frame, w.special_per_frame, w.heads, w.head_dim, w.block)
+    t0 = time.perf_counter()
+    Q, K = oracle.to_f64(x.q, w.dtype), oracle.to_f64(x.k, w.dtype)
+    PQ, PK = oracle.pool(Q, lay), oracle.pool(K, lay)
+    dens = None if x.scores is None else oracle.water_fill(x.scores, w.heads * (1 - w.rho), 1.0)
+    kh = oracle.head_k(lay, w.rho, dens)
+    m = oracle.predict_mask(PQ, PK, lay.head_dim, kh, w.tau)
+    t_mask = time.perf_counter() - t0
+    V = oracle.to_f64(x.v, w.dtype)
+    g = np.random.default_rng(seed)
+    pairs = [(int(g.integers(0, lay.heads)), int(g.integers(0, lay.B))) for _ in range(100000)]
+    t1 = time.perf_counter()
+    done = 0
+    sr = oracle.special_rows(lay)
+    for h, i in pairs:
+        rows = oracle.patch_rows(lay)[slice(*oracle.block_bounds(lay, i))]
+        keys = np.concatenate([sr, oracle.patch_keys_of(lay, m.selected[h, i])])
+        oracle.attend(Q[rows, h], K[keys, h], V[keys, h])
+        done += 1
+        if time.perf_counter() - t1 > budget_s * 0.8:
+            break
+    t_patch = time.perf_counter() - t1
+    t2 = time.perf_counter()
+    n_spec_rows = 0
+    if lay.Ns:
+        for h in range(lay.heads):
+            rows = sr[g.choice(len(sr), size=min(8, len(sr)), replace=False)]
+            oracle.attend(Q[rows, h], K[:, h], V[:, h])
+            n_spec_rows += len(rows)
+    t_spec = time.perf_counter() - t2
+    total_pairs = lay.heads * lay.B
+    est = t_mask + t_patch * total_pairs / done + (t_spec * (lay.heads * lay.Ns) / n_spec_rows if n_spec_rows else 0)
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    sample = (f"full pool+mask ({t_mask:.1f} s); attention of {done}/{total_pairs} (head, query-block) pairs "
+              f"({t_patch:.1f} s) and {n_spec_rows}/{lay.heads * lay.Ns} special (row, head) pairs "
+              f"({t_spec:.1f} s), scaled to one layer")
+    return est * 1e3, threads, sample
+
+
+def reference_arm(args, w):
+    x = synth.make_inputs(w)
+    times = []
+    for s in range(args.warmup + args.steps):
+        ms, threads, sample = oracle_layer_sample(w, x, budget_s=args.ref_budget, seed=s)
+        if s >= args.warmup:
+            times.append(ms)
+    v = float(np.mean(times))
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": v, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w),
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w):
+    return {"workload": f"{w.name}: {w.frames} frames x ({w.patch_per_frame} patch + {w.special_per_frame} special)"
+                        f" tokens, {w.heads} heads, d={w.head_dim}, b={w.block}, rho={w.rho}, tau={w.tau}"
+                        + (", per-head budgets (LogNormal(0,1) scores, capped water-filling, cap 1)"
+                           if w.head_budgets else ""),
+            "frames": w.frames, "tokens_per_frame": w.tokens_per_frame, "heads": w.heads, "head_dim": w.head_dim,
+            "block": w.block, "rho": w.rho, "tau": w.tau, "global_batch": 1, "seq_len": w.n_tokens,
+            "parallelism": "replicas",
+            "l2": "inputs larger than L2 (Q, K, V and the packed workspace: about 1 GB touched per step)"}
+
+
+# ---------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="perhead100", choices=sorted(configs.ALL))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--ref-budget", type=float, default=3.0, help="seconds of oracle work per reference step")
+    ap.add_argument("--dense-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    args = ap.parse_args()
+    w = configs.ALL[args.workload]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            reference_arm(args, w)
+        return
+    if args.warmup < 3:
+        args.warmup = 3
+
+    import torch
+    from view_transformers_b200 import _lib, layer
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    x = synth.make_inputs(w)
+    density = _lib.bsa_head_budgets(x.scores, w.rho, 1.0) if x.scores is not None else None
+    L = layer.BlockSparseLayer.for_workload(w, head_density=density)
+    q, k, v = (layer.to_device(a, w.dtype) for a in (x.q, x.k, x.v))
+
+    run_steps(torch, L, q, k, v, args.warmup)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        per_stage, total_ms = run_steps(torch, L, q, k, v, args.steps)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    status = L.check_status()
+    clocks = clk.summary()
+    t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+    if dist:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = total_ms / (args.steps * world)          # whole job: layers processed by all ranks
+
+    kv_cnt = L.buf.kv_cnt.cpu().numpy()
+    kv_idx = L.buf.kv_idx.cpu().numpy().view(np.uint16)
+    f_sparse = sparse_flops(kv_cnt, kv_idx, w)
+    f_special = special_flops(w)
+    density_real = f_sparse / (4 * w.head_dim * w.heads * float(w.n_patch) ** 2)
+    stage_ms = {k_: float(np.mean(vs)) for k_, vs in per_stage.items()}
+
+    # dense comparator: the same kernels with every block kept
+    Ld = layer.BlockSparseLayer.for_workload(w.with_(rho=0.0, tau=0.0, head_budgets=False))
+    run_steps(torch, Ld, q, k, v, 2)
+    dense_stage, dense_total = run_steps(torch, Ld, q, k, v, args.dense_steps)
+    dense_ms = dense_total / args.dense_steps
+    del Ld
+
+    # end to end through the public API: pinned host inputs in, output back to the host
+    hq, hk, hv = (t_.cpu().pin_memory() for t_ in (q, k, v))
+    hout = torch.empty(L.buf.out.shape, dtype=L.buf.out.dtype).pin_memory()
+    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def e2e_step():
+        qd.copy_(hq, non_blocking=True)
+        kd.copy_(hk, non_blocking=True)
+        vd.copy_(hv, non_blocking=True)
+        out = L.forward(qd, kd, vd)
+        hout.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record()
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    s1.record()
+    s1.synchronize()
+    e2e_ms = s0.elapsed_time(s1) / args.e2e_steps
+    t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+    if dist:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_value = float(t.item()) / world
+    h2d = 3 * q.numel() * q.element_size()
+    d2h = hout.numel() * hout.element_size()
+
+    hbm, tf_burst, tf_sus, peak_src = peaks()
+    sparse_ms = stage_ms["sparse"]
+    achieved = f_sparse / (sparse_ms * 1e-3) / 1e12
+    sb = stage_bytes(w)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded N(0,1) Q/K/V, 5% planted correspondences)",
+        "config": workload_config(w),
+        "effective_tflops": (f_sparse + f_special) / (ms_per_step * 1e-3) / 1e12,
+        "sparse_kernel_tflops": achieved,
+        "dense_ms_per_layer": dense_ms, "speedup_vs_dense": dense_ms / ms_per_step,
+        "density": density_real, "sparsity": 1 - density_real,
+        "stage_ms": stage_ms, "dense_stage_ms": {k_: float(np.mean(vs)) for k_, vs in dense_stage.items()},
+        "mask_prediction_gbs": sb["pool"] / ((stage_ms["pool"] + stage_ms["mask"]) * 1e-3) / 1e9,
+        "roofline": {"kernel": "bsa_block_sparse_attn (tcgen05 attention, sparse mode)", "bound": "tensor",
+                     "achieved": achieved, "peak": tf_sus, "unit": "TFLOP/s", "frac": achieved / tf_sus,
+                     "peak_kind": f"{peak_src} sustained bf16 (kernel timed inside back-to-back layers)",
+                     "frac_of_burst": achieved / tf_burst, "frac_of_nominal_2250": achieved / 2250.0,
+                     "flops_per_launch": f_sparse, "traffic": None},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": sum(LAUNCHES_PER_STEP.values()) * args.steps,
+        "clocks": clocks, "device_status": status,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        ms, threads, sample = oracle_layer_sample(w, x, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": ms, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

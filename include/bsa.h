@@ -1,0 +1,209 @@
+/*
+ * bsa.h -- C ABI of the block-sparse global attention layer for multi-view geometry
+ * transformers, built for NVIDIA B200 (sm_100a).
+ *
+ * The layer and its five steps are those of "Block-Sparse Global Attention for
+ * Efficient Multi-View Geometry Transformers" (CVPR 2026 paper notes):
+ *   - 方法详解 / 整体框架 (flowchart): split the special tokens X_s from the patch
+ *     tokens X_p; predict a block mask on X_p; block-sparse attention on the selected
+ *     Q-K blocks; dense attention for X_s; merge the outputs;
+ *   - 关键设计 1: average pooling P_b(Q), P_b(K) by block size b, softmax of
+ *     P_b(Q) P_b(K)^T; Eq. (1) dense attention; Eq. (2) masked attention;
+ *   - 关键设计 2: Top-K + CDF dual threshold with k = floor(B (1 - rho));
+ *   - 关键设计 3: the 1 camera + 4 register tokens of each frame stay dense.
+ * Per-head budgets follow "HeSS: Head Sensitivity Score for Sparsity Redistribution
+ * in VGGT", 提案手法 (iterative capped redistribution of the layer budget).
+ *
+ * Conventions for every call:
+ *   - Token layout: Q, K, V and out are row-major [N, H, d] with N = F * T tokens
+ *     (frame-major), row stride H * d elements. The first S tokens of each frame are
+ *     the special tokens; the remaining P = T - S are patch tokens. The patch tokens
+ *     of all frames, concatenated in frame order, form X_p with Np = F * P rows; patch
+ *     token p (0 <= p < Np) is row (p / P) * T + S + (p % P).
+ *   - Blocks: block j covers patch tokens [j b, min((j+1) b, Np)); B = ceil(Np / b).
+ *     Blocks may straddle frames; the last block may be short (ragged).
+ *   - Pointers named *_dev or documented as device memory are CUDA device pointers;
+ *     host arrays are documented as such. The caller owns and allocates every buffer;
+ *     the library never allocates, frees or synchronises (except bsa_check_status).
+ *     Device pointers must be 16-byte aligned.
+ *   - Every device call is asynchronous and ordered on `stream` (NULL = legacy stream).
+ *   - status_dev: optional device int32 (NULL allowed). Kernels write the first device-
+ *     side error (BSA_ERR_TIMEOUT, BSA_ERR_DEVICE_BOUNDS) there and skip the faulty
+ *     access instead of faulting; read it with bsa_check_status. Zero it before use.
+ *   - Host-side validation happens before any launch; on error nothing is launched.
+ *     A failed launch returns BSA_ERR_CUDA.
+ */
+#ifndef BSA_H
+#define BSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BSA_API __attribute__((visibility("default")))
+#else
+#define BSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* bsa_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    BSA_OK = 0,
+    BSA_ERR_INVALID_ARG = 1,   /* null pointer, bad shape or value, misaligned pointer */
+    BSA_ERR_UNSUPPORTED = 2,   /* valid arguments outside what the kernels implement */
+    BSA_ERR_CUDA = 3,          /* a CUDA runtime or driver call failed */
+    BSA_ERR_TIMEOUT = 4,       /* device: a bounded wait ran out */
+    BSA_ERR_DEVICE_BOUNDS = 5  /* device: an out-of-range index was rejected */
+} bsa_status;
+
+typedef enum { BSA_F32 = 0, BSA_BF16 = 1 } bsa_dtype;
+
+typedef struct {
+    int32_t frames;            /* F >= 1 */
+    int32_t tokens_per_frame;  /* T = P + S, P >= 1 */
+    int32_t special_per_frame; /* S >= 0, prefix of every frame (1 camera + 4 register: 5) */
+    int32_t heads;             /* H >= 1 */
+    int32_t head_dim;          /* d; only 64 is implemented */
+    int32_t block;             /* b >= 1 */
+    bsa_dtype dtype;           /* element type of Q, K, V and out */
+} bsa_layout;
+
+/* Limits of the implementation (BSA_ERR_UNSUPPORTED beyond them). */
+#define BSA_HEAD_DIM 64
+#define BSA_MAX_BLOCKS 8192       /* B, bounded by the per-row selection buffer */
+#define BSA_MAX_HEADS 128
+#define BSA_F32_MAX_TOKENS 65536  /* f32 inputs run on CUDA cores; meant for small layers */
+
+/* ---------------------------------------------------------------------------------
+ * Step 1 -- block pooling P_b (关键设计 1).
+ * pq[h, j, :] = mean of Q[row(p), h, :] over the patch tokens p of block j (the
+ * divisor is the block's real token count); the same for pk from K.
+ *   q, k    : device, [N, H, d] of layout->dtype
+ *   pq, pk  : device, float32 [H, B, d]
+ */
+BSA_API bsa_status bsa_pool_qk(const bsa_layout* layout, const void* q, const void* k,
+                       float* pq, float* pk, int32_t* status_dev, bsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * Steps 2-3 -- pooled softmax and dual-threshold block selection (关键设计 1, 2).
+ * For every head h and query block i: s_ij = <pq[h,i], pk[h,j]> / sqrt(d),
+ * p_ij = softmax_j(s_ij); rank the blocks by p (descending, ties to the lower index),
+ * C(n) = cumulative mass of the first n; keep n = min(B, max(k_h, n_tau)) blocks where
+ * n_tau = min{n >= 1 : C(n) >= tau} (0 if tau <= 0, B if never reached).
+ * k_h = floor(B (1 - rho) + 1e-9) for every head when head_density is NULL; otherwise
+ * k_h = clamp(floor(B head_density[h] + 1e-9), 1, B) and rho only validates that
+ * sum_h head_density[h] = H (1 - rho) within 1e-9 * H.
+ *   pq, pk        : device, float32 [H, B, d] (from bsa_pool_qk)
+ *   rho, tau      : in [0, 1]
+ *   head_density  : host, double [H] in [0, 1], or NULL
+ *   mask_bits     : device, uint32 [H, B, ceil(B/32)] (bit j%32 of word j/32 = block j
+ *                   kept), or NULL
+ *   kv_idx        : device, uint16 [H, B, B]; row (h, i) holds the kept blocks in
+ *                   ascending order in its first kv_cnt[h, i] entries (rest untouched)
+ *   kv_cnt        : device, int32 [H, B]
+ */
+BSA_API bsa_status bsa_predict_mask(const bsa_layout* layout, const float* pq, const float* pk,
+                            double rho, double tau, const double* head_density,
+                            uint32_t* mask_bits, uint16_t* kv_idx, int32_t* kv_cnt,
+                            int32_t* status_dev, bsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * Packing (prepares steps 4 and 5 for bf16 layers; the token split of 关键设计 3 made
+ * physical). Copies the patch tokens and the special tokens of Q, K and V into a
+ * head-major workspace: per head, rows of d = 64 elements, patch rows padded to a
+ * multiple of 128 and special rows padded likewise, padding zeroed; Q and K stay bf16,
+ * V is converted to fp16 (the operand type of the P.V product; exact for |v| in
+ * [2^-14, 65504], smaller magnitudes lose precision, larger ones overflow).
+ * Must run after Q, K, V hold the layer's values and before bsa_block_sparse_attn /
+ * bsa_special_dense on the same stream. Not needed (no-op) for f32 layouts.
+ *   q, k, v          : device, [N, H, d] bf16
+ *   workspace        : device, at least bsa_workspace_size() bytes, 1024-byte aligned
+ */
+BSA_API bsa_status bsa_pack_qkv(const bsa_layout* layout, const void* q, const void* k, const void* v,
+                        void* workspace, size_t workspace_bytes, int32_t* status_dev,
+                        bsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * Step 4 -- block-sparse attention over the selected blocks (关键设计 1, Eq. (2)).
+ * For every head h and patch token p of query block i:
+ *   o_pp[p, h, :] = softmax over the patch keys of the blocks kv_idx[h, i, :kv_cnt[h,i]]
+ *                   of (q . k / sqrt(d)), times V;
+ *   lse_pp[h, p]  = ln sum exp(q . k / sqrt(d)) over those keys.
+ * Keys of unselected blocks are excluded (not zeroed). A row with no kept block gets
+ * o_pp = 0 and lse_pp = -inf. Block indices >= B are skipped and reported as
+ * BSA_ERR_DEVICE_BOUNDS through status_dev. Listed indices are expected to be distinct
+ * (as bsa_predict_mask writes them).
+ *   q, k, v   : device, [N, H, d] of layout->dtype (read directly for f32 layouts)
+ *   workspace : bf16 layouts: the packed copy written by bsa_pack_qkv (read only);
+ *               f32 layouts: ignored (may be NULL)
+ *   kv_idx, kv_cnt : device, as written by bsa_predict_mask
+ *   o_pp      : device, float32 [Np, H, d];  lse_pp : device, float32 [H, Np]
+ * bf16 runs on the tensor cores (tcgen05 MMA, TMEM accumulators, TMA tile loads, P in
+ * fp16) and needs block in {64, 128}; f32 runs on CUDA cores in fp32.
+ */
+BSA_API bsa_status bsa_block_sparse_attn(const bsa_layout* layout, const void* q, const void* k,
+                                 const void* v, const void* workspace, size_t workspace_bytes,
+                                 const uint16_t* kv_idx, const int32_t* kv_cnt,
+                                 float* o_pp, float* lse_pp, int32_t* status_dev,
+                                 bsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * Step 5 -- dense path of the special tokens (关键设计 3).
+ *   (i)  every special token attends over all N tokens: out[special rows] (final);
+ *   (ii) every patch token attends over the Ns = F * S special tokens:
+ *        o_ps[p, h, :] and lse_ps[h, p] (as for step 4; -inf and 0 when S = 0).
+ *   q, k, v   : device, [N, H, d] of layout->dtype (read directly for f32 layouts)
+ *   workspace : bf16: the packed copy written by bsa_pack_qkv; f32: ignored (may be NULL)
+ *   out       : device, [N, H, d] of layout->dtype; only the special rows are written
+ *   o_ps    : device, float32 [Np, H, d], or NULL to skip (ii) (lse_ps then ignored)
+ *   lse_ps  : device, float32 [H, Np]
+ */
+BSA_API bsa_status bsa_special_dense(const bsa_layout* layout, const void* q, const void* k,
+                             const void* v, const void* workspace, size_t workspace_bytes,
+                             void* out, float* o_ps, float* lse_ps, int32_t* status_dev,
+                             bsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * Step 6 -- merge (flowchart "合并输出"): one softmax over the special keys and the
+ * selected patch keys, assembled exactly from the two partial results:
+ *   L = ln(exp(lse_pp) + exp(lse_ps));
+ *   out[row(p), h, :] = exp(lse_pp - L) o_pp[p, h, :] + exp(lse_ps - L) o_ps[p, h, :].
+ * Rows where both lse are -inf get 0.
+ *   o_pp, o_ps : device, float32 [Np, H, d];  lse_pp, lse_ps : device, float32 [H, Np]
+ *   out        : device, [N, H, d] of layout->dtype; only the patch rows are written
+ */
+BSA_API bsa_status bsa_merge(const bsa_layout* layout, const float* o_pp, const float* lse_pp,
+                     const float* o_ps, const float* lse_ps, void* out,
+                     int32_t* status_dev, bsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
+ * Host helpers (no device work).
+ */
+/* B = ceil(F P / b). */
+BSA_API bsa_status bsa_num_blocks(const bsa_layout* layout, int32_t* num_blocks);
+/* Bytes of the packed workspace of bsa_pack_qkv (0 for f32 layouts). */
+BSA_API bsa_status bsa_workspace_size(const bsa_layout* layout, size_t* bytes);
+/* k = floor(B (1 - rho) + 1e-9), rho in [0, 1]. */
+BSA_API bsa_status bsa_k_from_rho(int32_t num_blocks, double rho, int32_t* k);
+/* k = clamp(floor(B density + 1e-9), 1, B), density in [0, 1]. */
+BSA_API bsa_status bsa_k_from_density(int32_t num_blocks, double density, int32_t* k);
+/* Capped redistribution of the layer budget H (1 - rho) across heads in proportion to
+ * positive scores (HeSS 提案手法): repeat d_h = (budget - cap #capped) s_h / sum of the
+ * uncapped s, capping every head above `cap`, until no new head is capped.
+ *   scores : host double [H] > 0;  density : host double [H] (output)
+ *   needs H (1 - rho) <= H cap. */
+BSA_API bsa_status bsa_head_budgets(const double* scores, int32_t heads, double rho, double cap,
+                            double* density);
+/* Waits for `stream`, reads *status_dev into the returned code and resets it to 0. */
+BSA_API bsa_status bsa_check_status(int32_t* status_dev, bsa_stream_t stream);
+BSA_API const char* bsa_status_string(bsa_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSA_H */

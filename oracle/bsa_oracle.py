@@ -113,13 +113,14 @@ def block_bounds(lay: Layout, j: int) -> tuple[int, int]:
 def pool(X: np.ndarray, lay: Layout) -> np.ndarray:
     """P_b(X): mean of each block of b consecutive patch tokens, per head [BSGA 关键设计 1].
 
-    X is [N, H, d] float64; returns [H, B, d].
+    X is [N, H, d] holding exact values (float32 or float64); sums are taken in float64.
+    Returns [H, B, d] float64.
     """
     Xp = X[patch_rows(lay)]
     out = np.zeros((lay.heads, lay.B, lay.head_dim))
     for j in range(lay.B):
         lo, hi = block_bounds(lay, j)
-        out[:, j, :] = Xp[lo:hi].sum(axis=0) / (hi - lo)
+        out[:, j, :] = Xp[lo:hi].sum(axis=0, dtype=np.float64) / (hi - lo)
     return out
 
 
@@ -262,6 +263,44 @@ def layer_forward(Q, K, V, lay: Layout, selected: np.ndarray, heads=None, qblock
             rows = pr[slice(*block_bounds(lay, i))]
             keys = np.concatenate([sr, patch_keys_of(lay, selected[h, i])])
             out[rows, h], _ = attend(Q[rows, h], K[keys, h], V[keys, h])
+    return out
+
+
+def allowed_keys(lay: Layout, selected: np.ndarray, h: int, row: int) -> np.ndarray:
+    """Token-level key mask [N] of query row `row` in head h: every key for a special
+    query; the special keys plus the patch keys of the kept blocks for a patch query."""
+    T, S = lay.tokens_per_frame, lay.special_per_frame
+    token = np.arange(lay.N)
+    is_special = (token % T) < S
+    if (row % T) < S:
+        return np.ones(lay.N, dtype=bool)
+    patch_index = (token // T) * lay.P + (token % T) - S          # valid where not special
+    i = ((row // T) * lay.P + (row % T) - S) // lay.block
+    kept = np.zeros(lay.N, dtype=bool)
+    kept[~is_special] = selected[h, i][patch_index[~is_special] // lay.block]
+    return is_special | kept
+
+
+def layer_rows(Q, K, V, lay: Layout, selected: np.ndarray, rows, heads, chunk: int = 32):
+    """Layer output for the (row, head) pairs only: the same keys as layer_forward, with
+    excluded keys removed from the softmax. Q, K, V hold exact values (float32/float64);
+    returns [len(rows), d] float64."""
+    rows = np.asarray(rows)
+    heads = np.asarray(heads)
+    out = np.empty((len(rows), lay.head_dim))
+    for h in np.unique(heads):
+        sel_pairs = np.nonzero(heads == h)[0]
+        Kh = K[:, h, :].astype(np.float64)
+        Vh = V[:, h, :].astype(np.float64)
+        for c in range(0, len(sel_pairs), chunk):
+            idx = sel_pairs[c:c + chunk]
+            q = Q[rows[idx], h, :].astype(np.float64)
+            s = q @ Kh.T / math.sqrt(lay.head_dim)
+            for a, r in enumerate(rows[idx]):
+                s[a, ~allowed_keys(lay, selected, int(h), int(r))] = -np.inf
+            m = s.max(axis=1, keepdims=True)
+            e = np.exp(s - m)
+            out[idx] = (e @ Vh) / e.sum(axis=1)[:, None]
     return out
 
 

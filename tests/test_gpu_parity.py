@@ -1,0 +1,166 @@
+"""GPU parity: every step of the layer, through the C ABI on cuda:0, against the fp64 oracle.
+
+Tolerances (from the acceptance rule of the layer): block masks bit-exact except blocks
+whose pooled-probability gap to the cut (or whose CDF crossing) is below 1e-6; outputs
+within relative L2 2e-3 and max-abs 2e-2 for bf16 inputs, 1e-5 for f32 inputs. Pooled
+means are fp32 sums of at most b values: within 1e-5 absolute.
+Full-size workloads are checked on 2,048 seeded (row, head) samples of the output, the
+mask on every row."""
+import numpy as np
+import pytest
+
+import oracle
+from oracle.compare import compare_mask, max_abs, nmse_per_head, rel_l2
+from view_transformers_b200 import configs
+
+from gpu_common import exact, head_density, inputs, oracle_layout, run_gpu, sample_pairs
+
+pytestmark = pytest.mark.gpu
+
+BF16_TOL = (2e-3, 2e-2)
+F32_TOL = (1e-5, 1e-5)
+
+SMALL_BF16 = [
+    configs.VGGT518.with_(name="vggt518_f3", frames=3, heads=4),
+    configs.SWEEP_TAU0.with_(name="sweep_tau0_f4", frames=4, heads=3),
+    configs.PERHEAD100.with_(name="perhead_f3", frames=3, heads=4, head_budgets=False, rho=0.6),
+]
+FULL = [configs.TINY, configs.TINY_TAU0, configs.VGGT518, configs.SWEEP_R50, configs.SWEEP_R75,
+        configs.SWEEP_R90, configs.SWEEP_TAU0, configs.PERHEAD100, configs.PERHEAD100_TAU95]
+
+
+def _oracle_mask(w, x, res):
+    lay = oracle_layout(w)
+    Q, K = exact(x.q, w.dtype), exact(x.k, w.dtype)
+    PQ, PK = oracle.pool(Q, lay), oracle.pool(K, lay)
+    dens = head_density(w, x)
+    kh = oracle.head_k(lay, w.rho, dens)
+    return lay, PQ, PK, kh, oracle.predict_mask(PQ, PK, lay.head_dim, kh, w.tau)
+
+
+def _check_lists(res, B):
+    """kv_idx rows are ascending, distinct, and agree with the mask bits and counts."""
+    sel, idx, cnt = res["selected"], res["kv_idx"], res["kv_cnt"]
+    assert np.array_equal(sel.sum(axis=2), cnt)
+    H = sel.shape[0]
+    for h in range(H):
+        for i in range(0, B, max(1, B // 64)):
+            lst = idx[h, i, :cnt[h, i]]
+            assert np.all(np.diff(lst.astype(np.int64)) > 0)
+            assert np.array_equal(np.nonzero(sel[h, i])[0], lst)
+
+
+@pytest.mark.parametrize("w", FULL + SMALL_BF16, ids=lambda w: w.name)
+def test_mask_and_layer(w):
+    x = inputs(w)
+    dens = head_density(w, x)
+    res = run_gpu(w, x, dens)
+    assert res["status"] == 0
+    lay, PQ, PK, kh, om = _oracle_mask(w, x, res)
+    # pooling
+    assert max_abs(res["pq"], PQ) < 1e-5 and max_abs(res["pk"], PK) < 1e-5
+    # mask
+    rep = compare_mask(om, res["selected"], w.tau)
+    print(f"{w.name}: mask rows {rep.rows} exact {rep.exact} exempt {rep.exempt} failed {rep.failed}")
+    assert rep.ok, rep.failures
+    assert np.all(res["kv_cnt"] >= np.minimum(kh, lay.B)[:, None])
+    _check_lists(res, lay.B)
+    # output, against the oracle fed the device mask
+    Q, K, V = (exact(a, w.dtype) for a in (x.q, x.k, x.v))
+    tol = F32_TOL if w.dtype == "f32" else BF16_TOL
+    if lay.N * lay.heads <= 4096:
+        ref = oracle.layer_forward(Q.astype(np.float64), K.astype(np.float64), V.astype(np.float64),
+                                   lay, res["selected"])
+        got = res["out"]
+        print(f"{w.name}: nmse/head {nmse_per_head(got, ref)}")
+    else:
+        rows, heads = sample_pairs(w, 2048)
+        ref = oracle.layer_rows(Q, K, V, lay, res["selected"], rows, heads)
+        got = res["out"][rows, heads]
+    e2, ea = rel_l2(got, ref), max_abs(got, ref)
+    print(f"{w.name}: rel_l2 {e2:.3e} max_abs {ea:.3e}")
+    assert e2 <= tol[0] and ea <= tol[1]
+
+
+@pytest.mark.parametrize("w", SMALL_BF16 + [configs.TINY], ids=lambda w: w.name)
+def test_partials(w):
+    """o_pp / lse_pp (kept patch keys) and o_ps / lse_ps (special keys) element by element."""
+    x = inputs(w)
+    res = run_gpu(w, x, head_density(w, x))
+    lay = oracle_layout(w)
+    Q, K, V = (exact(a, w.dtype).astype(np.float64) for a in (x.q, x.k, x.v))
+    o_pp, l_pp, o_ps, l_ps = oracle.partials(Q, K, V, lay, res["selected"])
+    tol = 1e-5 if w.dtype == "f32" else 2e-3
+    for got, ref in ((res["o_pp"], o_pp), (res["o_ps"], o_ps)):
+        assert rel_l2(got, ref) <= tol
+    assert max_abs(res["lse_pp"], l_pp) < 1e-4 and max_abs(res["lse_ps"], l_ps) < 1e-4
+
+
+@pytest.mark.slow
+def test_long500_mask_full_and_sampled_rows():
+    w = configs.LONG500
+    x = inputs(w)
+    res = run_gpu(w, x)
+    assert res["status"] == 0
+    lay, PQ, PK, kh, om = _oracle_mask(w, x, res)
+    assert max_abs(res["pq"], PQ) < 1e-5
+    rep = compare_mask(om, res["selected"], w.tau)
+    print(f"long500: mask rows {rep.rows} exact {rep.exact} exempt {rep.exempt} failed {rep.failed}")
+    assert rep.ok, rep.failures
+    rows, heads = sample_pairs(w, 2048)
+    Q, K, V = (exact(a, w.dtype) for a in (x.q, x.k, x.v))
+    ref = oracle.layer_rows(Q, K, V, lay, res["selected"], rows, heads)
+    got = res["out"][rows, heads]
+    assert rel_l2(got, ref) <= BF16_TOL[0] and max_abs(got, ref) <= BF16_TOL[1]
+
+
+# ------------------------------------------------------------------ edge cases
+
+EDGE = [
+    configs.Workload("no_special", 3, 777, 0, 2, 64, 128, 0.5, 0.5, "bf16", "five_percent"),
+    configs.Workload("empty_lists", 3, 777, 5, 2, 64, 128, 1.0, 0.0, "bf16", "five_percent"),
+    configs.Workload("one_block", 1, 100, 5, 2, 64, 128, 0.5, 0.5, "bf16", "five_percent"),
+    configs.Workload("b64_odd_tail", 3, 777, 5, 2, 64, 64, 0.7, 0.0, "bf16", "five_percent"),
+    configs.Workload("dense_rho0", 2, 300, 5, 2, 64, 64, 0.0, 0.0, "bf16", "five_percent"),
+    configs.Workload("f32_ragged", 3, 37, 4, 2, 64, 10, 0.6, 0.3, "f32", "tiny"),
+    configs.Workload("f32_no_special", 2, 40, 0, 2, 64, 16, 0.5, 0.5, "f32", "tiny"),
+]
+
+
+@pytest.mark.parametrize("w", EDGE, ids=lambda w: w.name)
+def test_edge_cases(w):
+    x = inputs(w)
+    res = run_gpu(w, x)
+    assert res["status"] == 0
+    lay, PQ, PK, kh, om = _oracle_mask(w, x, res)
+    assert compare_mask(om, res["selected"], w.tau).ok
+    Q, K, V = (exact(a, w.dtype).astype(np.float64) for a in (x.q, x.k, x.v))
+    if w.name == "empty_lists":
+        assert res["kv_cnt"].max() == 0
+        assert np.all(res["lse_pp"] == -np.inf) and np.all(res["o_pp"] == 0)
+    if w.name == "dense_rho0":
+        assert res["selected"].all()
+    ref = oracle.layer_forward(Q, K, V, lay, res["selected"])
+    tol = F32_TOL if w.dtype == "f32" else BF16_TOL
+    assert rel_l2(res["out"], ref) <= tol[0] and max_abs(res["out"], ref) <= tol[1]
+
+
+def test_out_of_range_block_index_is_reported_not_faulted():
+    w = configs.VGGT518.with_(name="tamper", frames=2, heads=2)
+    x = inputs(w)
+
+    def tamper(L):
+        import torch
+        L.buf.kv_idx[0, 0, 0] = 30000          # >= B: must be skipped and reported
+        torch.cuda.synchronize()
+
+    res = run_gpu(w, x, tamper=tamper)
+    assert res["status"] == 5                   # BSA_ERR_DEVICE_BOUNDS
+    assert np.isfinite(res["out"]).all()
+
+
+def test_deterministic():
+    w = SMALL_BF16[0]
+    x = inputs(w)
+    a, b = run_gpu(w, x), run_gpu(w, x)
+    assert np.array_equal(a["out"], b["out"]) and np.array_equal(a["selected"], b["selected"])

@@ -335,3 +335,19 @@ def test_mask_comparison_rule_accepts_near_ties_only():
     wrong = np.zeros((1, 1, 4), dtype=bool); wrong[0, 0, 2] = True          # far from the cut
     assert compare_mask(m, wrong, 0.0).failed == 1
     assert compare_mask(m, sel[None], 0.0).exact == 1
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_layer_rows_match_layer_forward(seed):
+    rng = np.random.default_rng(seed)
+    lay = _rand_layout(rng, H=3, d=8, S=int(rng.integers(1, 6)))
+    Q, K, V = (rng.standard_normal((lay.N, 3, 8)) for _ in range(3))
+    sel = rng.random((3, lay.B, lay.B)) < 0.5
+    full = oracle.layer_forward(Q, K, V, lay, sel)
+    rows = rng.integers(0, lay.N, 40)
+    heads = rng.integers(0, 3, 40)
+    got = oracle.layer_rows(Q.astype(np.float32), K.astype(np.float32), V.astype(np.float32), lay, sel,
+                            rows, heads)
+    Q, K, V = (x.astype(np.float32).astype(np.float64) for x in (Q, K, V))
+    full = oracle.layer_forward(Q, K, V, lay, sel)
+    assert np.allclose(got, full[rows, heads], atol=1e-12)

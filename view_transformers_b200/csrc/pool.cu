@@ -1,0 +1,96 @@
+// Block average pooling P_b of Q and K ("Block-Sparse Global Attention for Efficient
+// Multi-View Geometry Transformers", 关键设计 1): the mean of each run of b consecutive
+// patch tokens of the concatenated patch sequence, per head, accumulated in fp32.
+//
+// HBM-bound: every patch row of Q and K is read once (Np * H * d elements each), the
+// pooled [H, B, d] fp32 tensors are written once. One CTA per (block, Q|K); each warp
+// reads whole 16-byte chunks of consecutive rows (a row holds all heads, 2 KB in bf16
+// at H = 16), so every load is a coalesced 512-byte warp transaction. Row groups inside
+// the CTA keep 8-16 independent 16-byte loads in flight per thread.
+#include "common.cuh"
+
+namespace bsa {
+namespace {
+
+constexpr int kPoolThreads = 256;
+
+template <typename T>
+__global__ void __launch_bounds__(kPoolThreads)
+pool_kernel(Geo g, const T* __restrict__ q, const T* __restrict__ k, float* __restrict__ pq,
+            float* __restrict__ pk) {
+    extern __shared__ float red[];  // [ngroups][per_round * V] partial sums
+    constexpr int V = Vec16<T>::n;
+    const int j = blockIdx.x;
+    const T* src = blockIdx.y == 0 ? q : k;
+    float* dst = blockIdx.y == 0 ? pq : pk;
+    const int row_elems = g.H * g.d;
+    const int chunks = row_elems / V;                     // 16-byte chunks per row
+    const int per_round = min(chunks, kPoolThreads);      // chunks covered per round
+    const int ngroups = kPoolThreads / per_round;         // row groups per round
+    const int lo = j * g.b;
+    const int hi = min(lo + g.b, g.Np);
+    const float count = (float)(hi - lo);
+    const int gi = threadIdx.x / per_round;
+    const int ci = threadIdx.x % per_round;
+
+    for (int c0 = 0; c0 < chunks; c0 += per_round) {
+        const int c = c0 + ci;
+        if (gi < ngroups && c < chunks) {
+            float acc[V];
+#pragma unroll
+            for (int e = 0; e < V; ++e) acc[e] = 0.f;
+            int p = lo + gi;
+            for (; p + 3 * ngroups < hi; p += 4 * ngroups) {   // four independent loads in flight
+                float x[4][V];
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    Vec16<T>::load(src + (size_t)patch_row(g, p + u * ngroups) * row_elems + c * V, x[u]);
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int e = 0; e < V; ++e) acc[e] += x[u][e];
+            }
+            for (; p < hi; p += ngroups) {
+                float x[V];
+                Vec16<T>::load(src + (size_t)patch_row(g, p) * row_elems + c * V, x);
+#pragma unroll
+                for (int e = 0; e < V; ++e) acc[e] += x[e];
+            }
+            float* r = red + (size_t)gi * per_round * V + ci * V;
+#pragma unroll
+            for (int e = 0; e < V; ++e) r[e] = acc[e];
+        }
+        __syncthreads();
+        const int width = min(per_round, chunks - c0) * V;
+        for (int e = threadIdx.x; e < width; e += kPoolThreads) {
+            float s = 0.f;
+            for (int gg = 0; gg < ngroups; ++gg) s += red[(size_t)gg * per_round * V + e];
+            const int el = c0 * V + e;
+            const int h = el / g.d;
+            const int dd = el - h * g.d;
+            dst[((size_t)h * g.B + j) * g.d + dd] = s / count;
+        }
+        __syncthreads();
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_pool(const Geo& g, bsa_dtype dt, const void* q, const void* k, float* pq,
+                        float* pk, cudaStream_t st) {
+    const int V = dt == BSA_BF16 ? 8 : 4;
+    const int chunks = g.H * g.d / V;
+    const int per_round = chunks < kPoolThreads ? chunks : kPoolThreads;
+    const size_t smem = (size_t)(kPoolThreads / per_round) * per_round * V * sizeof(float);
+    const dim3 grid(g.B, 2);
+    if (dt == BSA_BF16) {
+        pool_kernel<__nv_bfloat16><<<grid, kPoolThreads, smem, st>>>(
+            g, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), pq, pk);
+    } else {
+        pool_kernel<float><<<grid, kPoolThreads, smem, st>>>(
+            g, static_cast<const float*>(q), static_cast<const float*>(k), pq, pk);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace bsa

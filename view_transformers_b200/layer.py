@@ -1,0 +1,124 @@
+"""Runs one block-sparse global-attention layer through the C ABI.
+
+Torch provides the device buffers and the stream; each step is one library call:
+  pool -> predict mask -> pack -> special dense -> block-sparse attention -> merge.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+
+_TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+@dataclass
+class Buffers:
+    pq: torch.Tensor
+    pk: torch.Tensor
+    mask_bits: torch.Tensor
+    kv_idx: torch.Tensor
+    kv_cnt: torch.Tensor
+    workspace: torch.Tensor
+    o_pp: torch.Tensor
+    lse_pp: torch.Tensor
+    o_ps: torch.Tensor
+    lse_ps: torch.Tensor
+    out: torch.Tensor
+    status: torch.Tensor
+
+
+class BlockSparseLayer:
+    """One global-attention layer of fixed geometry and selection hyper-parameters."""
+
+    def __init__(self, frames: int, tokens_per_frame: int, special_per_frame: int, heads: int,
+                 head_dim: int, block: int, dtype: str, rho: float, tau: float, head_density=None,
+                 device: str | torch.device = "cuda"):
+        self.layout = _lib.make_layout(frames, tokens_per_frame, special_per_frame, heads, head_dim, block, dtype)
+        self.dtype = dtype
+        self.rho, self.tau = float(rho), float(tau)
+        self.head_density = None if head_density is None else [float(x) for x in head_density]
+        self.device = torch.device(device)
+        self.B = _lib.bsa_num_blocks(self.layout)
+        self.ws_bytes = _lib.bsa_workspace_size(self.layout)
+        F, T, S, H, d = frames, tokens_per_frame, special_per_frame, heads, head_dim
+        self.N, self.Np, self.H, self.d = F * T, F * (T - S), H, d
+        B, dev = self.B, self.device
+        words = (B + 31) // 32
+        self.buf = Buffers(
+            pq=torch.empty((H, B, d), dtype=torch.float32, device=dev),
+            pk=torch.empty((H, B, d), dtype=torch.float32, device=dev),
+            mask_bits=torch.empty((H, B, words), dtype=torch.int32, device=dev),
+            kv_idx=torch.empty((H, B, B), dtype=torch.int16, device=dev),
+            kv_cnt=torch.empty((H, B), dtype=torch.int32, device=dev),
+            # 1024-byte alignment for the TMA tiles: over-allocate and offset
+            workspace=torch.empty(max(self.ws_bytes, 1) + 1024, dtype=torch.uint8, device=dev),
+            o_pp=torch.empty((self.Np, H, d), dtype=torch.float32, device=dev),
+            lse_pp=torch.empty((H, self.Np), dtype=torch.float32, device=dev),
+            o_ps=torch.empty((self.Np, H, d), dtype=torch.float32, device=dev),
+            lse_ps=torch.empty((H, self.Np), dtype=torch.float32, device=dev),
+            out=torch.empty((self.N, H, d), dtype=_TORCH_DTYPE[dtype], device=dev),
+            status=torch.zeros(1, dtype=torch.int32, device=dev),
+        )
+        base = self.buf.workspace.data_ptr()
+        self.ws_ptr = (base + 1023) // 1024 * 1024 if self.ws_bytes else 0
+
+    @classmethod
+    def for_workload(cls, w, head_density=None, device="cuda") -> "BlockSparseLayer":
+        return cls(w.frames, w.tokens_per_frame, w.special_per_frame, w.heads, w.head_dim, w.block,
+                   w.dtype, w.rho, w.tau, head_density, device)
+
+    # individual steps -------------------------------------------------------------
+    def predict(self, q: torch.Tensor, k: torch.Tensor, stream: int | None = None) -> None:
+        st = self._stream(stream)
+        b = self.buf
+        _lib.bsa_pool_qk(self.layout, q.data_ptr(), k.data_ptr(), b.pq.data_ptr(), b.pk.data_ptr(),
+                         b.status.data_ptr(), st)
+        _lib.bsa_predict_mask(self.layout, b.pq.data_ptr(), b.pk.data_ptr(), self.rho, self.tau,
+                              self.head_density, b.mask_bits.data_ptr(), b.kv_idx.data_ptr(),
+                              b.kv_cnt.data_ptr(), b.status.data_ptr(), st)
+
+    def attend(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream: int | None = None) -> torch.Tensor:
+        st = self._stream(stream)
+        b = self.buf
+        qp, kp, vp = q.data_ptr(), k.data_ptr(), v.data_ptr()
+        _lib.bsa_pack_qkv(self.layout, qp, kp, vp, self.ws_ptr, self.ws_bytes, b.status.data_ptr(), st)
+        _lib.bsa_special_dense(self.layout, qp, kp, vp, self.ws_ptr, self.ws_bytes, b.out.data_ptr(),
+                               b.o_ps.data_ptr(), b.lse_ps.data_ptr(), b.status.data_ptr(), st)
+        _lib.bsa_block_sparse_attn(self.layout, qp, kp, vp, self.ws_ptr, self.ws_bytes, b.kv_idx.data_ptr(),
+                                   b.kv_cnt.data_ptr(), b.o_pp.data_ptr(), b.lse_pp.data_ptr(),
+                                   b.status.data_ptr(), st)
+        _lib.bsa_merge(self.layout, b.o_pp.data_ptr(), b.lse_pp.data_ptr(), b.o_ps.data_ptr(),
+                       b.lse_ps.data_ptr(), b.out.data_ptr(), b.status.data_ptr(), st)
+        return b.out
+
+    def forward(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream: int | None = None) -> torch.Tensor:
+        """The whole layer: [N, H, d] tensors in the layer dtype, on this device."""
+        self.predict(q, k, stream)
+        return self.attend(q, k, v, stream)
+
+    def check_status(self, stream: int | None = None) -> int:
+        return _lib.bsa_check_status(self.buf.status.data_ptr(), self._stream(stream))
+
+    # helpers ----------------------------------------------------------------------
+    def _stream(self, stream):
+        return torch.cuda.current_stream(self.device).cuda_stream if stream is None else stream
+
+    def selected(self):
+        """Kept-block mask [H, B, B] (numpy bool, host) from the mask bits."""
+        import numpy as np
+        words = self.buf.mask_bits.cpu().numpy().view(np.uint32)
+        bits = np.unpackbits(words.view(np.uint8), axis=-1, bitorder="little")
+        return bits[..., :self.B].astype(bool)
+
+
+def to_device(x, dtype: str, device="cuda") -> torch.Tensor:
+    """Storage array from synth (uint16 bf16 bits or float32) -> device tensor of the layer dtype."""
+    import numpy as np
+    if dtype == "bf16":
+        t = torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16)
+    else:
+        t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    return t.to(device)
