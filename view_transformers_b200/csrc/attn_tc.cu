@@ -77,6 +77,7 @@ struct Ctl {
     uint64_t s_full[2];
     uint64_t p_full[2];
     uint64_t o_done;
+    uint64_t o_final;
     uint64_t drain;
     int meta_nvalid[NS];
     uint32_t meta_member[NS];
@@ -137,6 +138,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(&ctl.p_full[b], 4);
         }
         mbar_init(&ctl.o_done, 1);
+        mbar_init(&ctl.o_final, 1);
         mbar_init(&ctl.drain, 1);
         ctl.n_tiles = 0;
         ctl.abort = 0;
@@ -273,6 +275,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                            (t > 0 || ks > 0) ? 1u : 0u);
                 mma_commit(&ctl.kv_empty[stage]);
                 mma_commit(&ctl.o_done);
+                if (t == n - 1) mma_commit(&ctl.o_final);
                 if (t + 2 < n) {
                     if (!mbar_wait(&ctl.o_done, t & 1, abort, prm.status)) break;   // P_t consumed
                     ok = issue_qk(t + 2);
@@ -352,7 +355,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         float o[64];
 #pragma unroll
         for (int c = 0; c < 64; ++c) o[c] = 0.f;
-        if (ok && n > 0 && warp_wait(&ctl.o_done, (n - 1) & 1, abort, prm.status, lane)) {
+        // A parity wait only tells apart phases within one of the barrier's current phase.
+        // Here o_done may still be two phases behind (tile n-1 done by this warp, P.V of
+        // tile n-2 still running), so the epilogue waits on its own single-phase barrier.
+        if (ok && n > 0 && warp_wait(&ctl.o_final, 0, abort, prm.status, lane)) {
             tc_fence_after();
             uint32_t r[2][32];
             tmem_ld32(lane_base + kColO, r[0]);
