@@ -31,7 +31,6 @@ from view_transformers_b200 import configs, synth  # noqa: E402
 
 METRIC = "global-attn ms/layer & effective TFLOPS vs dense at 100 frames, rho=0.75"
 UNIT = "ms/layer"
-STAGES = ["pool", "mask", "pack", "special", "sparse", "merge"]
 
 
 def peaks():
@@ -96,6 +95,24 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------- helpers
+def measured_traffic(w, path):
+    """DRAM bytes per launch of the fused kernel from the committed ncu record, scaled to this
+    workload by patch tokens x heads; None when the kernel source changed since the capture."""
+    import hashlib
+    if path != "fused":
+        return None
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "fused_traffic.json")))
+        src = b"".join(open(os.path.join(ROOT, "view_transformers_b200", "csrc", f), "rb").read()
+                       for f in ("attn_tc.cu", "sm100.cuh", "tc_layout.cuh"))
+    except (OSError, ValueError):
+        return None
+    if hashlib.sha256(src).hexdigest() != rec.get("source_sha256"):
+        return None
+    return rec["dram_bytes_per_launch"] * (w.n_patch * w.heads) / (rec["patch_tokens"] * rec["heads"])
+
+
+
 def sparse_flops(kv_cnt, kv_idx, w) -> float:
     """4 d sum_h sum_(i, j kept) |I_i| |J_j| over patch query/key blocks."""
     B, b, Np = w.n_blocks, w.block, w.n_patch
@@ -121,45 +138,62 @@ def stage_bytes(w) -> dict:
     }
 
 
-def run_steps(torch, L, q, k, v, steps, record_stages=True):
-    """Runs `steps` layers; returns per-step stage durations (ms) and the total (ms)."""
+def step_calls(L, q, k, v, path: str):
+    """The library calls of one layer, as (stage name, callable, our kernel launches)."""
+    from view_transformers_b200 import _lib
+    import torch
+    b = L.buf
+    sp = torch.cuda.current_stream().cuda_stream
+    status = b.status.data_ptr()
+    lay = L.layout
+    qp, kp, vp = q.data_ptr(), k.data_ptr(), v.data_ptr()
+    calls = [
+        ("pool", lambda: _lib.bsa_pool_qk(lay, qp, kp, b.pq.data_ptr(), b.pk.data_ptr(), status, sp), 1),
+        ("mask", lambda: _lib.bsa_predict_mask(lay, b.pq.data_ptr(), b.pk.data_ptr(), L.rho, L.tau, L.head_density,
+                                               b.mask_bits.data_ptr(), b.kv_idx.data_ptr(), b.kv_cnt.data_ptr(),
+                                               status, sp), 1),
+        ("pack", lambda: _lib.bsa_pack_qkv(lay, qp, kp, vp, L.ws_ptr, L.ws_bytes, status, sp), 1),
+    ]
+    if path == "fused":
+        calls += [
+            ("special", lambda: _lib.bsa_special_dense(lay, qp, kp, vp, L.ws_ptr, L.ws_bytes, b.out.data_ptr(),
+                                                       None, None, status, sp), 2),
+            ("sparse", lambda: _lib.bsa_block_sparse_attn_fused(lay, qp, kp, vp, L.ws_ptr, L.ws_bytes,
+                                                                b.kv_idx.data_ptr(), b.kv_cnt.data_ptr(),
+                                                                b.out.data_ptr(), status, sp), 1),
+        ]
+    else:
+        calls += [
+            ("special", lambda: _lib.bsa_special_dense(lay, qp, kp, vp, L.ws_ptr, L.ws_bytes, b.out.data_ptr(),
+                                                       b.o_ps.data_ptr(), b.lse_ps.data_ptr(), status, sp), 3),
+            ("sparse", lambda: _lib.bsa_block_sparse_attn(lay, qp, kp, vp, L.ws_ptr, L.ws_bytes, b.kv_idx.data_ptr(),
+                                                          b.kv_cnt.data_ptr(), b.o_pp.data_ptr(),
+                                                          b.lse_pp.data_ptr(), status, sp), 1),
+            ("merge", lambda: _lib.bsa_merge(lay, b.o_pp.data_ptr(), b.lse_pp.data_ptr(), b.o_ps.data_ptr(),
+                                             b.lse_ps.data_ptr(), b.out.data_ptr(), status, sp), 1),
+        ]
+    return calls
+
+
+def run_steps(torch, L, q, k, v, steps, path="fused"):
+    """Runs `steps` layers; returns per-stage durations (ms, per step) and the total (ms)."""
     st = torch.cuda.current_stream()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)] for _ in range(steps)]
+    calls = step_calls(L, q, k, v, path)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(steps)]
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
-    b = L.buf
-    from view_transformers_b200 import _lib
-    sp = st.cuda_stream
-    status = b.status.data_ptr()
     start.record(st)
     for s in range(steps):
         e = evs[s]
         e[0].record(st)
-        _lib.bsa_pool_qk(L.layout, q.data_ptr(), k.data_ptr(), b.pq.data_ptr(), b.pk.data_ptr(), status, sp)
-        e[1].record(st)
-        _lib.bsa_predict_mask(L.layout, b.pq.data_ptr(), b.pk.data_ptr(), L.rho, L.tau, L.head_density,
-                              b.mask_bits.data_ptr(), b.kv_idx.data_ptr(), b.kv_cnt.data_ptr(), status, sp)
-        e[2].record(st)
-        _lib.bsa_pack_qkv(L.layout, q.data_ptr(), k.data_ptr(), v.data_ptr(), L.ws_ptr, L.ws_bytes, status, sp)
-        e[3].record(st)
-        _lib.bsa_special_dense(L.layout, q.data_ptr(), k.data_ptr(), v.data_ptr(), L.ws_ptr, L.ws_bytes,
-                               b.out.data_ptr(), b.o_ps.data_ptr(), b.lse_ps.data_ptr(), status, sp)
-        e[4].record(st)
-        _lib.bsa_block_sparse_attn(L.layout, q.data_ptr(), k.data_ptr(), v.data_ptr(), L.ws_ptr, L.ws_bytes,
-                                   b.kv_idx.data_ptr(), b.kv_cnt.data_ptr(), b.o_pp.data_ptr(),
-                                   b.lse_pp.data_ptr(), status, sp)
-        e[5].record(st)
-        _lib.bsa_merge(L.layout, b.o_pp.data_ptr(), b.lse_pp.data_ptr(), b.o_ps.data_ptr(), b.lse_ps.data_ptr(),
-                       b.out.data_ptr(), status, sp)
-        e[6].record(st)
+        for i, (_, fn, _) in enumerate(calls):
+            fn()
+            e[i + 1].record(st)
     end.record(st)
     end.synchronize()
     per_stage = {name: [evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(steps)]
-                 for i, name in enumerate(STAGES)}
-    return per_stage, start.elapsed_time(end)
-
-
-LAUNCHES_PER_STEP = {"pool": 1, "mask": 1, "pack": 1, "special": 2, "sparse": 1, "merge": 1}
+                 for i, (name, _, _) in enumerate(calls)}
+    return per_stage, start.elapsed_time(end), sum(c[2] for c in calls)
 
 
 # ---------------------------------------------------------------------------- CPU oracle
@@ -250,8 +284,15 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=3.0, help="seconds of oracle work per reference step")
     ap.add_argument("--dense-steps", type=int, default=3)
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--frames", type=int, default=None,
+                    help="override the workload's frame count (smaller cases for profiling)")
+    ap.add_argument("--path", default=None, choices=["fused", "five"],
+                    help="fused: special dense + one fused patch-row pass (bf16 default); "
+                         "five: the five-step path with fp32 partials and the merge")
     args = ap.parse_args()
     w = configs.ALL[args.workload]
+    if args.frames:
+        w = w.with_(name=f"{w.name}_f{args.frames}", frames=args.frames)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -272,18 +313,19 @@ def main():
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
 
+    path = args.path or ("fused" if w.dtype == "bf16" else "five")
     x = synth.make_inputs(w)
     density = _lib.bsa_head_budgets(x.scores, w.rho, 1.0) if x.scores is not None else None
     L = layer.BlockSparseLayer.for_workload(w, head_density=density)
     q, k, v = (layer.to_device(a, w.dtype) for a in (x.q, x.k, x.v))
 
-    run_steps(torch, L, q, k, v, args.warmup)
+    run_steps(torch, L, q, k, v, args.warmup, path)
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
-        per_stage, total_ms = run_steps(torch, L, q, k, v, args.steps)
+        per_stage, total_ms, launches = run_steps(torch, L, q, k, v, args.steps, path)
         torch.cuda.synchronize()
     if dist:
         dist.barrier()
@@ -305,44 +347,51 @@ def main():
     stage_ms = {k_: float(np.mean(vs)) for k_, vs in per_stage.items()}
 
     # dense comparator: the same kernels with every block kept
-    Ld = layer.BlockSparseLayer.for_workload(w.with_(rho=0.0, tau=0.0, head_budgets=False))
-    run_steps(torch, Ld, q, k, v, 2)
-    dense_stage, dense_total = run_steps(torch, Ld, q, k, v, args.dense_steps)
-    dense_ms = dense_total / args.dense_steps
-    del Ld
+    dense_ms, dense_stage = None, {}
+    if args.dense_steps > 0:
+        Ld = layer.BlockSparseLayer.for_workload(w.with_(rho=0.0, tau=0.0, head_budgets=False))
+        run_steps(torch, Ld, q, k, v, 2, path)
+        dense_stage, dense_total, _ = run_steps(torch, Ld, q, k, v, args.dense_steps, path)
+        dense_ms = dense_total / args.dense_steps
+        del Ld
 
     # end to end through the public API: pinned host inputs in, output back to the host
-    hq, hk, hv = (t_.cpu().pin_memory() for t_ in (q, k, v))
-    hout = torch.empty(L.buf.out.shape, dtype=L.buf.out.dtype).pin_memory()
-    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    e2e_ms = float("nan")
+    h2d = 3 * q.numel() * q.element_size()
+    d2h = L.buf.out.numel() * L.buf.out.element_size()
+    if args.e2e_steps > 0:
+        hq, hk, hv = (t_.cpu().pin_memory() for t_ in (q, k, v))
+        hout = torch.empty(L.buf.out.shape, dtype=L.buf.out.dtype).pin_memory()
+        qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
 
-    def e2e_step():
-        qd.copy_(hq, non_blocking=True)
-        kd.copy_(hk, non_blocking=True)
-        vd.copy_(hv, non_blocking=True)
-        out = L.forward(qd, kd, vd)
-        hout.copy_(out, non_blocking=True)
+        def e2e_step():
+            qd.copy_(hq, non_blocking=True)
+            kd.copy_(hk, non_blocking=True)
+            vd.copy_(hv, non_blocking=True)
+            out = L.forward(qd, kd, vd, fused=(path == "fused"))
+            hout.copy_(out, non_blocking=True)
 
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s0.record()
-    for _ in range(args.e2e_steps):
-        e2e_step()
-    s1.record()
-    s1.synchronize()
-    e2e_ms = s0.elapsed_time(s1) / args.e2e_steps
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        s1.record()
+        s1.synchronize()
+        e2e_ms = s0.elapsed_time(s1) / args.e2e_steps
     t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
     if dist:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     e2e_value = float(t.item()) / world
-    h2d = 3 * q.numel() * q.element_size()
-    d2h = hout.numel() * hout.element_size()
 
     hbm, tf_burst, tf_sus, peak_src = peaks()
     sparse_ms = stage_ms["sparse"]
-    achieved = f_sparse / (sparse_ms * 1e-3) / 1e12
+    # algorithmic work of the timed sparse kernel: kept patch-patch entries, plus the
+    # patch-to-special entries when the special keys are fused into it
+    f_kernel = f_sparse + (4.0 * w.head_dim * w.heads * w.n_patch * w.n_special if path == "fused" else 0.0)
+    achieved = f_kernel / (sparse_ms * 1e-3) / 1e12
     sb = stage_bytes(w)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -351,17 +400,20 @@ def main():
         "config": workload_config(w),
         "effective_tflops": (f_sparse + f_special) / (ms_per_step * 1e-3) / 1e12,
         "sparse_kernel_tflops": achieved,
-        "dense_ms_per_layer": dense_ms, "speedup_vs_dense": dense_ms / ms_per_step,
+        "dense_ms_per_layer": dense_ms, "speedup_vs_dense": dense_ms / ms_per_step if dense_ms else None,
         "density": density_real, "sparsity": 1 - density_real,
         "stage_ms": stage_ms, "dense_stage_ms": {k_: float(np.mean(vs)) for k_, vs in dense_stage.items()},
         "mask_prediction_gbs": sb["pool"] / ((stage_ms["pool"] + stage_ms["mask"]) * 1e-3) / 1e9,
-        "roofline": {"kernel": "bsa_block_sparse_attn (tcgen05 attention, sparse mode)", "bound": "tensor",
+        "path": path,
+        "roofline": {"kernel": ("bsa_block_sparse_attn_fused" if path == "fused" else "bsa_block_sparse_attn")
+                               + " (tcgen05 attention)", "bound": "tensor",
                      "achieved": achieved, "peak": tf_sus, "unit": "TFLOP/s", "frac": achieved / tf_sus,
                      "peak_kind": f"{peak_src} sustained bf16 (kernel timed inside back-to-back layers)",
                      "frac_of_burst": achieved / tf_burst, "frac_of_nominal_2250": achieved / 2250.0,
-                     "flops_per_launch": f_sparse, "traffic": None},
+                     "flops_per_launch": f_kernel, "traffic": measured_traffic(w, path),
+                     "traffic_unit": "bytes per launch (ncu dram read+write, scaled by patch tokens x heads)"},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": sum(LAUNCHES_PER_STEP.values()) * args.steps,
+        "gpu_launches": launches * args.steps,
         "clocks": clocks, "device_status": status,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

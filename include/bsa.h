@@ -181,6 +181,22 @@ BSA_API bsa_status bsa_merge(const bsa_layout* layout, const float* o_pp, const 
                      int32_t* status_dev, bsa_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
+ * Steps 4, 5(ii) and 6 in one pass (bf16 only): for every patch token p of query block i
+ * and head h, out[row(p), h, :] = one softmax over the special keys and the patch keys of
+ * the kept blocks kv_idx[h, i, :kv_cnt[h, i]] -- the same result as bsa_block_sparse_attn
+ * + bsa_special_dense (ii) + bsa_merge, without the fp32 partials. The special rows of out
+ * are not touched (bsa_special_dense with o_ps = NULL writes them).
+ *   q, k, v   : unused (the packed copies in workspace are read); may be NULL
+ *   workspace : the packed copy written by bsa_pack_qkv
+ *   out       : device, [N, H, d] bf16
+ */
+BSA_API bsa_status bsa_block_sparse_attn_fused(const bsa_layout* layout, const void* q, const void* k,
+                                               const void* v, const void* workspace,
+                                               size_t workspace_bytes, const uint16_t* kv_idx,
+                                               const int32_t* kv_cnt, void* out,
+                                               int32_t* status_dev, bsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
  * Host helpers (no device work).
  */
 /* B = ceil(F P / b). */

@@ -43,8 +43,15 @@ def run_gpu(w: configs.Workload, x: synth.LayerInputs, density=None, tamper=None
     torch.cuda.synchronize()
     status = L.check_status()
     out = L.buf.out.float().cpu().numpy()
+    out_fused = None
+    if w.dtype == "bf16":
+        L.buf.out.zero_()
+        L.attend_fused(q, k, v)
+        torch.cuda.synchronize()
+        status = status or L.check_status()
+        out_fused = L.buf.out.float().cpu().numpy()
     res = dict(
-        layer=L, status=status, out=out, selected=L.selected(),
+        layer=L, status=status, out=out, out_fused=out_fused, selected=L.selected(),
         kv_idx=L.buf.kv_idx.cpu().numpy().view(np.uint16), kv_cnt=L.buf.kv_cnt.cpu().numpy(),
         pq=L.buf.pq.cpu().numpy(), pk=L.buf.pk.cpu().numpy(),
         o_pp=L.buf.o_pp.cpu().numpy(), lse_pp=L.buf.lse_pp.cpu().numpy(),

@@ -73,8 +73,8 @@ def test_perhead_budgets(lib):
 def test_workspace_size(lib):
     w = configs.PERHEAD100
     n = _lib.bsa_workspace_size(_lib.layout_of(w))
-    np_pad, ns_pad = 77824, 512
-    assert n == 3 * 16 * (np_pad + ns_pad) * 128
+    np_pad, ns_pad, nsplit = 77824, 512, 10        # key-range splits: ceil((4 + 608) / 64)
+    assert n == 3 * 16 * (np_pad + ns_pad) * 128 + nsplit * 16 * ns_pad * (64 + 1) * 4
     assert _lib.bsa_workspace_size(_lib.layout_of(configs.TINY)) == 0
 
 

@@ -40,6 +40,7 @@ _SIGS = {
     "bsa_block_sparse_attn": [_LP, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp, _vp, _i32p, _st],
     "bsa_special_dense": [_LP, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp, _i32p, _st],
     "bsa_merge": [_LP, _vp, _vp, _vp, _vp, _vp, _i32p, _st],
+    "bsa_block_sparse_attn_fused": [_LP, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp, _i32p, _st],
     "bsa_num_blocks": [_LP, ctypes.POINTER(ctypes.c_int32)],
     "bsa_workspace_size": [_LP, ctypes.POINTER(ctypes.c_size_t)],
     "bsa_k_from_rho": [ctypes.c_int32, ctypes.c_double, ctypes.POINTER(ctypes.c_int32)],
@@ -167,3 +168,9 @@ def bsa_special_dense(layout, q, k, v, workspace, workspace_bytes, out, o_ps, ls
 
 def bsa_merge(layout, o_pp, lse_pp, o_ps, lse_ps, out, status=0, stream=0) -> None:
     _check("bsa_merge", load().bsa_merge(ctypes.byref(layout), o_pp, lse_pp, o_ps, lse_ps, out, status, stream))
+
+
+def bsa_block_sparse_attn_fused(layout, q, k, v, workspace, workspace_bytes, kv_idx, kv_cnt, out, status=0,
+                                stream=0) -> None:
+    _check("bsa_block_sparse_attn_fused", load().bsa_block_sparse_attn_fused(
+        ctypes.byref(layout), q, k, v, workspace, workspace_bytes, kv_idx, kv_cnt, out, status, stream))

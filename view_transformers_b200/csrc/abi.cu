@@ -288,6 +288,25 @@ bsa_status bsa_special_dense(const bsa_layout* layout, const void* q, const void
     return from_cuda(e);
 }
 
+bsa_status bsa_block_sparse_attn_fused(const bsa_layout* layout, const void* q, const void* k, const void* v,
+                                       const void* workspace, size_t workspace_bytes, const uint16_t* kv_idx,
+                                       const int32_t* kv_cnt, void* out, int32_t* status_dev,
+                                       bsa_stream_t stream) {
+    (void)q;
+    (void)k;
+    (void)v;
+    Geo g;
+    bsa_status s = make_geo(layout, &g);
+    if (s != BSA_OK) return s;
+    if (layout->dtype != BSA_BF16 || !tc_supported(g)) return BSA_ERR_UNSUPPORTED;
+    if (!kv_idx || !kv_cnt || !out || !aligned16(out) || !aligned16(kv_idx) || !aligned16(kv_cnt))
+        return BSA_ERR_INVALID_ARG;
+    s = check_ws(g, workspace, workspace_bytes);
+    if (s != BSA_OK) return s;
+    return from_cuda(launch_attn_tc(g, 3, workspace, kv_idx, kv_cnt, nullptr, nullptr, out, status_dev,
+                                    reinterpret_cast<cudaStream_t>(stream)));
+}
+
 bsa_status bsa_merge(const bsa_layout* layout, const float* o_pp, const float* lse_pp,
                      const float* o_ps, const float* lse_ps, void* out, int32_t* status_dev,
                      bsa_stream_t stream) {

@@ -1,26 +1,42 @@
 // Tensor-core attention for the bf16 layer on B200 (sm_100a): tcgen05 MMA with TMEM
-// accumulators, TMA tile loads, fp32 online softmax. It covers the three attention pieces
-// of "Block-Sparse Global Attention for Efficient Multi-View Geometry Transformers":
+// accumulators, TMA tile loads, fp32 online softmax. It covers the attention pieces of
+// "Block-Sparse Global Attention for Efficient Multi-View Geometry Transformers":
 //   MODE_SPARSE        patch query tile over the kept key blocks of its query blocks
 //                      (关键设计 1, Eq. (2); masked entries are excluded) -> o_pp, lse_pp
 //   MODE_PATCH_SPECIAL patch query tile over every special key (关键设计 3)  -> o_ps, lse_ps
-//   MODE_SPECIAL_ALL   special query tile over every key (关键设计 3)       -> out (bf16)
+//   MODE_SPECIAL_ALL   special query tile over one chunk of all keys (关键设计 3) -> split
+//                      partials in the workspace, combined by special_combine_kernel
+//   MODE_FUSED         patch query tile over the special keys and the kept key blocks in
+//                      one online softmax: steps 4, 5(ii) and the merge in one pass -> out
 //
 // Inputs come from the packed workspace (pack.cu): per head, 64-wide rows of 128 bytes,
-// so each query tile (128 rows) and each key tile (BKV = b rows, or 128) is one 2D TMA box
-// with the 128-byte swizzle that the MMA descriptors expect.
+// so each query tile (128 rows) and each key tile (BKV rows) is one 2D TMA box with the
+// 128-byte swizzle that the MMA descriptors expect.
 //
-// One CTA per (query tile, head), 6 warps:
+// One CTA per work item, two CTAs per SM (112 KB of shared memory and 256 TMEM columns
+// each, so the softmax of one CTA overlaps the tensor-core work of the other). 6 warps:
 //   warp 0      TMA producer: Q once, then K/V tiles into an NS-stage ring;
-//   warp 1      MMA issuer (one thread): S = Q K^T into one of two TMEM S buffers, and
-//               O += P V with P read from TMEM (fp16, written over its S buffer);
+//   warp 1      MMA issuer (one thread): S = Q K^T (TMEM columns [0,128)), then
+//               O += P V with P (fp16) read from TMEM columns [128,192), O in [192,256);
+//               the next S is computed as soon as the softmax has read the current one;
 //   warps 2..5  softmax, one query row per thread (TMEM lane = row): row max, lazy
 //               rescale of O (only when the running max grows by more than 2^8),
 //               p = 2^(s log2(e)/sqrt(d) - m) in fp32, P rounded to fp16 into TMEM,
 //               then the epilogue O / l and the log-sum-exp.
 // For b = 64 a 128-row query tile holds two query blocks; it walks the union of their
 // kept blocks, and each row ignores the key blocks its own query block did not keep.
-// Every mbarrier wait is bounded; a timeout is reported through the status word.
+//
+// Barrier protocol (u = tile index of the CTA). A parity wait only tells apart phases
+// within one of the barrier's current phase; every wait below has that property:
+//   kv_full[s]/kv_empty[s]  TMA ring; the producer refills a stage after P.V of its tile;
+//   s_full   QK^T of tile u done (commit; also implies every earlier MMA is done);
+//   s_free   all 4 softmax warps have S_u in registers (count 4) -> QK^T of tile u+1;
+//   p_full   all 4 softmax warps wrote P_u (count 4) -> P.V of tile u;
+//   o_done   P.V of tile u done (commit). The softmax waits o_done(u-1) before writing
+//            P_u or rescaling O: at tile u it has seen s_full(u), so P.V of tile u-2 is
+//            done and o_done is at most one phase behind;
+//   o_final  single phase, committed after the last P.V: the epilogue waits on it.
+// Every wait is bounded; a timeout is reported through the status word.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -36,16 +52,16 @@ namespace {
 
 using namespace sm100;
 
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0;
-constexpr uint32_t kColS1 = 128;
-constexpr uint32_t kColO = 256;
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColS = 0;
+constexpr uint32_t kColP = 128;
+constexpr uint32_t kColO = 192;
 constexpr float kScaleLog2 = 0.18033688011112042f;   // log2(e) / sqrt(64)
 constexpr float kRescale = 8.0f;                     // lazy-rescale threshold (log2 units)
 constexpr float kLn2 = 0.69314718055994531f;
 constexpr int kThreads = 192;
 
-enum { MODE_SPARSE = 0, MODE_PATCH_SPECIAL = 1, MODE_SPECIAL_ALL = 2 };
+enum { MODE_SPARSE = 0, MODE_PATCH_SPECIAL = 1, MODE_SPECIAL_ALL = 2, MODE_FUSED = 3 };
 
 struct TcParams {
     Geo g;
@@ -55,12 +71,15 @@ struct TcParams {
     float* o_part;
     float* lse_part;
     __nv_bfloat16* out;
+    float* spart;
+    float* slse;
     int32_t* status;
+    int q_tiles;   // query tiles per head
 };
 
 template <int BKV>
 struct Cfg {
-    static constexpr int NS = BKV == 128 ? 4 : 8;   // K/V stages
+    static constexpr int NS = BKV == 128 ? 3 : 6;   // K/V stages
     static constexpr int QB = 128 / BKV;            // query blocks per 128-row query tile
     static constexpr uint32_t kTileBytes = BKV * 128;
     static constexpr uint32_t kOffQ = 0;
@@ -74,8 +93,9 @@ struct Ctl {
     uint64_t q_full;
     uint64_t kv_full[NS];
     uint64_t kv_empty[NS];
-    uint64_t s_full[2];
-    uint64_t p_full[2];
+    uint64_t s_full;
+    uint64_t s_free;
+    uint64_t p_full;
     uint64_t o_done;
     uint64_t o_final;
     uint64_t drain;
@@ -87,9 +107,9 @@ struct Ctl {
 };
 
 template <int BKV>
-constexpr size_t smem_bytes() {
-    return Cfg<BKV>::kOffCtl + ((sizeof(Ctl<Cfg<BKV>::NS>) + 15) / 16 * 16) +
-           (size_t)Cfg<BKV>::QB * (BSA_MAX_BLOCKS / 32) * 4 + 1024;
+size_t smem_bytes(int num_blocks) {
+    const size_t words = (size_t)(num_blocks + 31) / 32;
+    return Cfg<BKV>::kOffCtl + (sizeof(Ctl<Cfg<BKV>::NS>) + 15) / 16 * 16 + Cfg<BKV>::QB * words * 4;
 }
 
 // Lane 0 waits, the whole warp gets the same answer (keeps .sync.aligned tcgen05 ops uniform).
@@ -106,25 +126,51 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity, int32
 }
 
 template <int MODE, int BKV>
-__global__ void __launch_bounds__(kThreads, 1)
-attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k0,
-               const __grid_constant__ CUtensorMap tm_v0, const __grid_constant__ CUtensorMap tm_k1,
-               const __grid_constant__ CUtensorMap tm_v1, const TcParams prm) {
+__global__ void __launch_bounds__(kThreads, 2)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ka,
+               const __grid_constant__ CUtensorMap tm_va, const __grid_constant__ CUtensorMap tm_kb,
+               const __grid_constant__ CUtensorMap tm_vb, const TcParams prm) {
     using C = Cfg<BKV>;
     constexpr int NS = C::NS;
     constexpr int QB = C::QB;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    constexpr uint32_t kAll = (1u << QB) - 1u;
+    constexpr bool kUnion = MODE == MODE_SPARSE || MODE == MODE_FUSED;   // walks kept blocks
+    extern __shared__ __align__(1024) uint8_t smem[];
     Ctl<NS>& ctl = *reinterpret_cast<Ctl<NS>*>(smem + C::kOffCtl);
     uint32_t* bits = reinterpret_cast<uint32_t*>(smem + C::kOffCtl + (sizeof(Ctl<NS>) + 15) / 16 * 16);
     const Geo& g = prm.g;
     const PackedLayout& pl = prm.pl;
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
-    const int h = blockIdx.x % g.H;
-    const int tq = blockIdx.x / g.H;
     volatile int* abort = &ctl.abort;
     const int words = (g.B + 31) / 32;
+
+    // tile swizzles assume a 1024-byte aligned base; refuse to run otherwise
+    if ((smem_u32(smem) & 1023u) != 0u) {
+        if (threadIdx.x == 0) record_error(prm.status, BSA_ERR_DEVICE_BOUNDS);
+        return;
+    }
+
+    // work item: head-major order keeps one head's keys hot in L2
+    int h, tq, split = 0;
+    if (MODE == MODE_SPECIAL_ALL) {
+        const int per_head = prm.q_tiles * pl.nsplit;
+        h = blockIdx.x / per_head;
+        const int r = blockIdx.x - h * per_head;
+        tq = r / pl.nsplit;
+        split = r - tq * pl.nsplit;
+    } else {
+        h = blockIdx.x / prm.q_tiles;
+        tq = blockIdx.x - h * prm.q_tiles;
+    }
+    const int sp_tiles = (g.Ns + BKV - 1) / BKV;   // special key tiles (BKV rows)
+    int t_begin = 0, t_end = 0;                    // MODE_SPECIAL_ALL key-tile range
+    if (MODE == MODE_SPECIAL_ALL) {
+        const int n_all = sp_tiles + pl.np_pad / 128;
+        const int chunk = (n_all + pl.nsplit - 1) / pl.nsplit;
+        t_begin = min(n_all, split * chunk);
+        t_end = min(n_all, t_begin + chunk);
+    }
 
     // ------------------------------------------------------------------ setup
     if (threadIdx.x == 0) {
@@ -133,10 +179,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(&ctl.kv_full[s], 1);
             mbar_init(&ctl.kv_empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&ctl.s_full[b], 1);
-            mbar_init(&ctl.p_full[b], 4);
-        }
+        mbar_init(&ctl.s_full, 1);
+        mbar_init(&ctl.s_free, 4);
+        mbar_init(&ctl.p_full, 4);
         mbar_init(&ctl.o_done, 1);
         mbar_init(&ctl.o_final, 1);
         mbar_init(&ctl.drain, 1);
@@ -146,18 +191,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch(&tm_q);
-        tma_prefetch(&tm_k0);
-        tma_prefetch(&tm_v0);
-        if (MODE == MODE_SPECIAL_ALL) {
-            tma_prefetch(&tm_k1);
-            tma_prefetch(&tm_v1);
-        }
+        tma_prefetch(&tm_ka);
+        tma_prefetch(&tm_va);
+        tma_prefetch(&tm_kb);
+        tma_prefetch(&tm_vb);
     }
     if (warp == 1) {
         tmem_alloc(&ctl.tmem_base, kTmemCols);
         tmem_relinquish();
     }
-    if (MODE == MODE_SPARSE) {
+    if (kUnion) {
         for (int x = threadIdx.x; x < QB * words; x += kThreads) bits[x] = 0u;
         __syncthreads();
         for (int qb = 0; qb < QB; ++qb) {
@@ -187,10 +230,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ctl.tmem_base;
-    const int ns_tiles = (g.Ns + 127) / 128;
     const int n = MODE == MODE_SPARSE ? ctl.n_tiles
-                : MODE == MODE_PATCH_SPECIAL ? ns_tiles
-                : ns_tiles + (g.Np + 127) / 128;
+                : MODE == MODE_FUSED ? sp_tiles + ctl.n_tiles
+                : MODE == MODE_PATCH_SPECIAL ? sp_tiles
+                : t_end - t_begin;
     int issued = 0;   // K/V tiles whose loads the producer issued
 
     if (warp == 0) {
@@ -201,16 +244,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             tma_load_2d(smem + C::kOffQ, &tm_q, &ctl.q_full, 0, q_row0);
             int w = 0;
             uint32_t cur = 0;
-            if (MODE == MODE_SPARSE && words > 0)
+            if (kUnion && words > 0)
                 for (int qb = 0; qb < QB; ++qb) cur |= bits[qb * words];
-            for (int t = 0; t < n; ++t) {
-                const int stage = t % NS;
-                if (t >= NS && !mbar_wait(&ctl.kv_empty[stage], ((t / NS) - 1) & 1, abort, prm.status)) break;
+            for (int u = 0; u < n; ++u) {
+                const int stage = u % NS;
+                if (u >= NS && !mbar_wait(&ctl.kv_empty[stage], ((u / NS) - 1) & 1, abort, prm.status)) break;
                 int row0, nvalid;
-                uint32_t member = 1u;
-                const CUtensorMap* mk = &tm_k0;
-                const CUtensorMap* mv = &tm_v0;
-                if (MODE == MODE_SPARSE) {
+                uint32_t member = kAll;
+                bool special;
+                if (MODE == MODE_SPECIAL_ALL) {
+                    const int t = t_begin + u;
+                    special = t < sp_tiles;
+                    const int base = special ? t * 128 : (t - sp_tiles) * 128;
+                    row0 = (special ? h * pl.ns_pad : h * pl.np_pad) + base;
+                    nvalid = min(128, (special ? g.Ns : g.Np) - base);
+                } else if (MODE == MODE_PATCH_SPECIAL || (MODE == MODE_FUSED && u < sp_tiles)) {
+                    special = true;
+                    row0 = h * pl.ns_pad + u * BKV;
+                    nvalid = min(BKV, g.Ns - u * BKV);
+                } else {
+                    special = false;
                     while (cur == 0u && w + 1 < words) {
                         ++w;
                         for (int qb = 0; qb < QB; ++qb) cur |= bits[qb * words + w];
@@ -223,22 +276,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     for (int qb = 0; qb < QB; ++qb) member |= ((bits[qb * words + w] >> bit) & 1u) << qb;
                     row0 = h * pl.np_pad + j * BKV;
                     nvalid = min(BKV, g.Np - j * BKV);
-                } else if (MODE == MODE_PATCH_SPECIAL || t < ns_tiles) {
-                    row0 = h * pl.ns_pad + t * 128;
-                    nvalid = min(128, g.Ns - t * 128);
-                } else {
-                    const int u = t - ns_tiles;
-                    row0 = h * pl.np_pad + u * 128;
-                    nvalid = min(128, g.Np - u * 128);
-                    mk = &tm_k1;
-                    mv = &tm_v1;
                 }
                 ctl.meta_nvalid[stage] = nvalid;
                 ctl.meta_member[stage] = member;
                 mbar_arrive_expect_tx(&ctl.kv_full[stage], 2 * C::kTileBytes);
-                tma_load_2d(smem + C::kOffK + stage * C::kTileBytes, mk, &ctl.kv_full[stage], 0, row0);
-                tma_load_2d(smem + C::kOffV + stage * C::kTileBytes, mv, &ctl.kv_full[stage], 0, row0);
-                issued = t + 1;
+                tma_load_2d(smem + C::kOffK + stage * C::kTileBytes, special ? &tm_ka : &tm_kb, &ctl.kv_full[stage],
+                            0, row0);
+                tma_load_2d(smem + C::kOffV + stage * C::kTileBytes, special ? &tm_va : &tm_vb, &ctl.kv_full[stage],
+                            0, row0);
+                issued = u + 1;
             }
             if (n == 0) drain_wait(&ctl.q_full, 0, prm.status);   // no MMA will consume Q
         }
@@ -248,38 +294,35 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             constexpr uint32_t idesc_qk = idesc_f16(128, BKV, 1u, false);
             constexpr uint32_t idesc_pv = idesc_f16(128, 64, 0u, true);
             const uint32_t q_base = smem_u32(smem + C::kOffQ);
-            auto issue_qk = [&](int t) -> bool {
-                const int stage = t % NS;
-                if (!mbar_wait(&ctl.kv_full[stage], (t / NS) & 1, abort, prm.status)) return false;
+            auto issue_qk = [&](int u) -> bool {
+                const int stage = u % NS;
+                if (!mbar_wait(&ctl.kv_full[stage], (u / NS) & 1, abort, prm.status)) return false;
                 tc_fence_after();
-                const uint32_t sbuf = tmem + ((t & 1) ? kColS1 : kColS0);
                 const uint32_t k_base = smem_u32(smem + C::kOffK + stage * C::kTileBytes);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_ss(sbuf, sdesc_sw128(q_base + 32 * ks, 16, 1024), sdesc_sw128(k_base + 32 * ks, 16, 1024),
-                           idesc_qk, ks > 0 ? 1u : 0u);
-                mma_commit(&ctl.s_full[t & 1]);
+                    mma_ss(tmem + kColS, sdesc_sw128(q_base + 32 * ks, 16, 1024),
+                           sdesc_sw128(k_base + 32 * ks, 16, 1024), idesc_qk, ks > 0 ? 1u : 0u);
+                mma_commit(&ctl.s_full);
                 return true;
             };
             bool ok = issue_qk(0);
-            if (ok && n > 1) ok = issue_qk(1);
-            for (int t = 0; ok && t < n; ++t) {
-                if (!mbar_wait(&ctl.p_full[t & 1], (t >> 1) & 1, abort, prm.status)) break;
+            for (int u = 0; ok && u < n; ++u) {
+                if (u + 1 < n) {
+                    if (!mbar_wait(&ctl.s_free, u & 1, abort, prm.status)) break;   // S_u read
+                    if (!issue_qk(u + 1)) break;
+                }
+                if (!mbar_wait(&ctl.p_full, u & 1, abort, prm.status)) break;
                 tc_fence_after();
-                const int stage = t % NS;
-                const uint32_t sbuf = tmem + ((t & 1) ? kColS1 : kColS0);
+                const int stage = u % NS;
                 const uint32_t v_base = smem_u32(smem + C::kOffV + stage * C::kTileBytes);
 #pragma unroll
                 for (int ks = 0; ks < BKV / 16; ++ks)
-                    mma_ts(tmem + kColO, sbuf + 8 * ks, sdesc_sw128(v_base + 2048 * ks, 0, 1024), idesc_pv,
-                           (t > 0 || ks > 0) ? 1u : 0u);
+                    mma_ts(tmem + kColO, tmem + kColP + 8 * ks, sdesc_sw128(v_base + 2048 * ks, 0, 1024), idesc_pv,
+                           (u > 0 || ks > 0) ? 1u : 0u);
                 mma_commit(&ctl.kv_empty[stage]);
                 mma_commit(&ctl.o_done);
-                if (t == n - 1) mma_commit(&ctl.o_final);
-                if (t + 2 < n) {
-                    if (!mbar_wait(&ctl.o_done, t & 1, abort, prm.status)) break;   // P_t consumed
-                    ok = issue_qk(t + 2);
-                }
+                if (u == n - 1) mma_commit(&ctl.o_final);
             }
         }
     } else {
@@ -287,109 +330,129 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int quad = warp & 3;
         const int row = quad * 32 + lane;
         const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-        const int row_qb = row / BKV;
+        const int row_qb = row / BKV;          // warp-uniform: a warp's 32 rows share a block
         float m_ref = -INFINITY;
         float l = 0.f;
         bool ok = true;
-        for (int t = 0; t < n; ++t) {
-            const int stage = t % NS;
-            if (!warp_wait(&ctl.kv_full[stage], (t / NS) & 1, abort, prm.status, lane)) { ok = false; break; }
+        for (int u = 0; u < n; ++u) {
+            const int stage = u % NS;
+            if (!warp_wait(&ctl.kv_full[stage], (u / NS) & 1, abort, prm.status, lane)) { ok = false; break; }
             const int nvalid = ctl.meta_nvalid[stage];
             const bool member = ((ctl.meta_member[stage] >> row_qb) & 1u) != 0u;
-            if (!warp_wait(&ctl.s_full[t & 1], (t >> 1) & 1, abort, prm.status, lane)) { ok = false; break; }
+            const bool full = member && nvalid == BKV;
+            if (!warp_wait(&ctl.s_full, u & 1, abort, prm.status, lane)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t sbuf = lane_base + ((t & 1) ? kColS1 : kColS0);
             uint32_t s[BKV];
 #pragma unroll
             for (int c = 0; c < BKV / 32; ++c)
-                tmem_ld32(sbuf + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * c]));
+                tmem_ld32(lane_base + kColS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * c]));
             tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl.s_free);   // the next QK^T may overwrite S
             float mt = -INFINITY;
+            if (full) {
 #pragma unroll
-            for (int c = 0; c < BKV; ++c)
-                if (member && c < nvalid) mt = fmaxf(mt, __uint_as_float(s[c]));
+                for (int c = 0; c < BKV; ++c) mt = fmaxf(mt, __uint_as_float(s[c]));
+            } else if (member) {
+#pragma unroll
+                for (int c = 0; c < BKV; ++c)
+                    if (c < nvalid) mt = fmaxf(mt, __uint_as_float(s[c]));
+            }
             const float mt2 = mt * kScaleLog2;
             const bool need = mt2 > m_ref + kRescale;
             const bool corr = need && m_ref != -INFINITY;
             const float new_ref = need ? mt2 : m_ref;
-            if (__any_sync(0xffffffffu, corr)) {
-                const float factor = corr ? ex2_approx(m_ref - new_ref) : 1.f;
-                if (t > 0 && !warp_wait(&ctl.o_done, (t - 1) & 1, abort, prm.status, lane)) { ok = false; break; }
-                tc_fence_after();
-                uint32_t o[2][32];
-                tmem_ld32(lane_base + kColO, o[0]);
-                tmem_ld32(lane_base + kColO + 32, o[1]);
-                tmem_wait_ld();
-#pragma unroll
-                for (int a = 0; a < 2; ++a)
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) o[a][c] = __float_as_uint(__uint_as_float(o[a][c]) * factor);
-                tmem_st32(lane_base + kColO, o[0]);
-                tmem_st32(lane_base + kColO + 32, o[1]);
-                tmem_wait_st();
-                l *= factor;
-            }
+            const float factor = corr ? ex2_approx(m_ref - new_ref) : 1.f;
             m_ref = new_ref;
-            uint32_t pk[BKV / 2];
+            // p in fp32, packed to fp16 pairs in place: pair i lands in s[i], after s[2i],
+            // s[2i+1] were read
             float rs = 0.f;
+            if (full) {
 #pragma unroll
-            for (int c = 0; c < BKV; c += 2) {
-                const bool v0 = member && c < nvalid;
-                const bool v1 = member && c + 1 < nvalid;
-                const float p0 = v0 ? ex2_approx(fmaf(__uint_as_float(s[c]), kScaleLog2, -m_ref)) : 0.f;
-                const float p1 = v1 ? ex2_approx(fmaf(__uint_as_float(s[c + 1]), kScaleLog2, -m_ref)) : 0.f;
-                rs += p0 + p1;
-                const __half2 hp = __floats2half2_rn(p0, p1);
-                pk[c / 2] = *reinterpret_cast<const uint32_t*>(&hp);
+                for (int c = 0; c < BKV; c += 2) {
+                    const float p0 = ex2_approx(fmaf(__uint_as_float(s[c]), kScaleLog2, -m_ref));
+                    const float p1 = ex2_approx(fmaf(__uint_as_float(s[c + 1]), kScaleLog2, -m_ref));
+                    rs += p0 + p1;
+                    const __half2 hp = __floats2half2_rn(p0, p1);
+                    s[c / 2] = *reinterpret_cast<const uint32_t*>(&hp);
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < BKV; c += 2) {
+                    const float p0 =
+                        member && c < nvalid ? ex2_approx(fmaf(__uint_as_float(s[c]), kScaleLog2, -m_ref)) : 0.f;
+                    const float p1 =
+                        member && c + 1 < nvalid ? ex2_approx(fmaf(__uint_as_float(s[c + 1]), kScaleLog2, -m_ref)) : 0.f;
+                    rs += p0 + p1;
+                    const __half2 hp = __floats2half2_rn(p0, p1);
+                    s[c / 2] = *reinterpret_cast<const uint32_t*>(&hp);
+                }
             }
-            l += rs;
+            l = l * factor + rs;
+            // P.V of the previous tile must be done before O is rescaled or P overwritten
+            if (u > 0 && !warp_wait(&ctl.o_done, (u - 1) & 1, abort, prm.status, lane)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            if (__any_sync(0xffffffffu, corr)) {
+#pragma unroll
+                for (int a = 0; a < 2; ++a) {
+                    uint32_t o[32];
+                    tmem_ld32(lane_base + kColO + 32 * a, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * factor);
+                    tmem_st32(lane_base + kColO + 32 * a, o);
+                }
+            }
 #pragma unroll
             for (int c = 0; c < BKV / 64; ++c)
-                tmem_st32(sbuf + 32 * c, *reinterpret_cast<const uint32_t(*)[32]>(&pk[32 * c]));
+                tmem_st32(lane_base + kColP + 32 * c, *reinterpret_cast<const uint32_t(*)[32]>(&s[32 * c]));
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&ctl.p_full[t & 1]);
+            if (lane == 0) mbar_arrive(&ctl.p_full);
         }
         // ------------------------------------------------------------ epilogue
-        float o[64];
-#pragma unroll
-        for (int c = 0; c < 64; ++c) o[c] = 0.f;
-        // A parity wait only tells apart phases within one of the barrier's current phase.
-        // Here o_done may still be two phases behind (tile n-1 done by this warp, P.V of
-        // tile n-2 still running), so the epilogue waits on its own single-phase barrier.
-        if (ok && n > 0 && warp_wait(&ctl.o_final, 0, abort, prm.status, lane)) {
-            tc_fence_after();
-            uint32_t r[2][32];
-            tmem_ld32(lane_base + kColO, r[0]);
-            tmem_ld32(lane_base + kColO + 32, r[1]);
-            tmem_wait_ld();
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                o[c] = __uint_as_float(r[0][c]) * inv;
-                o[32 + c] = __uint_as_float(r[1][c]) * inv;
-            }
-        } else if (n > 0) {
-            l = 0.f;   // aborted: report an empty row
-        }
+        const bool have = ok && n > 0 && warp_wait(&ctl.o_final, 0, abort, prm.status, lane);
+        if (!have) l = 0.f;   // empty row, or aborted: report an empty row
+        const float inv = l > 0.f ? 1.f / l : 0.f;
         const float lse = l > 0.f ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
-        if (MODE == MODE_SPECIAL_ALL) {
-            const int ts = tq * 128 + row;
-            if (ts < g.Ns) {
-                __nv_bfloat16* dst = prm.out + (size_t)special_row(g, ts) * g.H * 64 + (size_t)h * 64;
+        if (have) tc_fence_after();
+        const int qrow = tq * 128 + row;
 #pragma unroll
-                for (int c = 0; c < 64; c += 8) Vec16<__nv_bfloat16>::store(dst + c, o + c);
+        for (int a = 0; a < 2; ++a) {
+            float o[32];
+            if (have) {
+                uint32_t r[32];
+                tmem_ld32(lane_base + kColO + 32 * a, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 32; ++c) o[c] = __uint_as_float(r[c]) * inv;
+            } else {
+#pragma unroll
+                for (int c = 0; c < 32; ++c) o[c] = 0.f;
             }
-        } else {
-            const int p = tq * 128 + row;
-            if (p < g.Np) {
-                float* dst = prm.o_part + ((size_t)p * g.H + h) * 64;
+            if (MODE == MODE_SPECIAL_ALL) {
+                float* dst = prm.spart + (((size_t)split * g.H + h) * pl.ns_pad + qrow) * 64 + 32 * a;
 #pragma unroll
-                for (int c = 0; c < 64; c += 4) Vec16<float>::store(dst + c, o + c);
-                prm.lse_part[(size_t)h * g.Np + p] = lse;
+                for (int c = 0; c < 32; c += 4) Vec16<float>::store(dst + c, o + c);
+            } else if (MODE == MODE_FUSED) {
+                if (qrow < g.Np) {
+                    __nv_bfloat16* dst = prm.out + (size_t)patch_row(g, qrow) * g.H * 64 + (size_t)h * 64 + 32 * a;
+#pragma unroll
+                    for (int c = 0; c < 32; c += 8) Vec16<__nv_bfloat16>::store(dst + c, o + c);
+                }
+            } else if (qrow < g.Np) {
+                float* dst = prm.o_part + ((size_t)qrow * g.H + h) * 64 + 32 * a;
+#pragma unroll
+                for (int c = 0; c < 32; c += 4) Vec16<float>::store(dst + c, o + c);
             }
         }
+        if (MODE == MODE_SPECIAL_ALL) prm.slse[((size_t)split * g.H + h) * pl.ns_pad + qrow] = lse;
+        else if (MODE != MODE_FUSED && qrow < g.Np) prm.lse_part[(size_t)h * g.Np + qrow] = lse;
     }
 
     // ------------------------------------------------------------------ teardown
@@ -397,8 +460,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (ctl.abort) {
         // let in-flight copies and MMAs land before the shared and tensor memory go away
         if (warp == 0 && lane == 0)
-            for (int t = max(0, issued - NS); t < issued; ++t)
-                drain_wait(&ctl.kv_full[t % NS], (t / NS) & 1, prm.status);
+            for (int u = max(0, issued - NS); u < issued; ++u)
+                drain_wait(&ctl.kv_full[u % NS], (u / NS) & 1, prm.status);
         if (warp == 1 && lane == 0) {
             mma_commit(&ctl.drain);
             drain_wait(&ctl.drain, 0, prm.status);
@@ -408,6 +471,40 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// Combines the key-range splits of the special queries: L = ln sum_s e^lse_s,
+// out = sum_s e^(lse_s - L) O_s, written to the special rows of out (bf16).
+__global__ void __launch_bounds__(256)
+special_combine_kernel(Geo g, PackedLayout pl, const float* __restrict__ spart, const float* __restrict__ slse,
+                       __nv_bfloat16* __restrict__ out) {
+    const size_t total = (size_t)g.Ns * g.H * 8;   // (special token, head, 8-element group)
+    for (size_t x = blockIdx.x * (size_t)blockDim.x + threadIdx.x; x < total;
+         x += (size_t)gridDim.x * blockDim.x) {
+        const int grp = (int)(x & 7);
+        const size_t th = x >> 3;
+        const int h = (int)(th % g.H);
+        const int t = (int)(th / g.H);
+        float mx = -INFINITY;
+        for (int s = 0; s < pl.nsplit; ++s) mx = fmaxf(mx, slse[((size_t)s * g.H + h) * pl.ns_pad + t]);
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        float wsum = 0.f;
+        if (mx != -INFINITY) {
+            for (int s = 0; s < pl.nsplit; ++s) {
+                const float w = expf(slse[((size_t)s * g.H + h) * pl.ns_pad + t] - mx);
+                wsum += w;
+                const float4* src =
+                    reinterpret_cast<const float4*>(spart + (((size_t)s * g.H + h) * pl.ns_pad + t) * 64 + grp * 8);
+                const float4 a = __ldg(src), b = __ldg(src + 1);
+                acc[0] += w * a.x; acc[1] += w * a.y; acc[2] += w * a.z; acc[3] += w * a.w;
+                acc[4] += w * b.x; acc[5] += w * b.y; acc[6] += w * b.z; acc[7] += w * b.w;
+            }
+        }
+        const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] *= inv;
+        Vec16<__nv_bfloat16>::store(out + (size_t)special_row(g, t) * g.H * 64 + (size_t)h * 64 + grp * 8, acc);
     }
 }
 
@@ -441,23 +538,26 @@ bool make_map(CUtensorMap* tm, const void* base, uint64_t rows, uint32_t box_row
 }
 
 template <int MODE, int BKV>
-cudaError_t launch_mode(const TcParams& prm, const CUtensorMap& q, const CUtensorMap& k0, const CUtensorMap& v0,
-                        const CUtensorMap& k1, const CUtensorMap& v1, int q_tiles, cudaStream_t st) {
-    const size_t smem = smem_bytes<BKV>();
+cudaError_t launch_mode(const TcParams& prm, const CUtensorMap& q, const CUtensorMap& ka, const CUtensorMap& va,
+                        const CUtensorMap& kb, const CUtensorMap& vb, int ctas, cudaStream_t st) {
+    if (ctas == 0) return cudaSuccess;
+    const size_t smem = smem_bytes<BKV>(prm.g.B);
     auto kern = attn_tc_kernel<MODE, BKV>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<q_tiles * prm.g.H, kThreads, smem, st>>>(q, k0, v0, k1, v1, prm);
+    kern<<<ctas, kThreads, smem, st>>>(q, ka, va, kb, vb, prm);
     return cudaGetLastError();
 }
 
 }  // namespace
 
+// mode: 0 sparse (o_part/lse_part), 1 patch->special (o_part/lse_part),
+//       2 special->all (out, through the split partials), 3 fused sparse + special keys (out)
 cudaError_t launch_attn_tc(const Geo& g, int mode, const void* ws, const uint16_t* kv_idx,
                            const int32_t* kv_cnt, float* o_part, float* lse_part, void* out,
                            int32_t* status, cudaStream_t st) {
     const PackedLayout pl = packed_layout(g);
-    const uint8_t* base = static_cast<const uint8_t*>(ws);
+    uint8_t* base = static_cast<uint8_t*>(const_cast<void*>(ws));
     TcParams prm;
     prm.g = g;
     prm.pl = pl;
@@ -466,29 +566,49 @@ cudaError_t launch_attn_tc(const Geo& g, int mode, const void* ws, const uint16_
     prm.o_part = o_part;
     prm.lse_part = lse_part;
     prm.out = static_cast<__nv_bfloat16*>(out);
+    prm.spart = reinterpret_cast<float*>(base + pl.spart);
+    prm.slse = reinterpret_cast<float*>(base + pl.slse);
     prm.status = status;
     const uint64_t prow = (uint64_t)g.H * pl.np_pad;
     const uint64_t srow = (uint64_t)g.H * pl.ns_pad;
-    CUtensorMap q, k0, v0, k1, v1;
-    if (mode == MODE_SPARSE) {
-        if (!make_map(&q, base + pl.qp, prow, 128, false) || !make_map(&k0, base + pl.kp, prow, g.b, false) ||
-            !make_map(&v0, base + pl.vp, prow, g.b, true))
+    const bool has_sp = g.Ns > 0;
+    CUtensorMap q, ka, va, kb, vb;
+    const int patch_tiles = pl.np_pad / 128;
+    if (mode == MODE_SPARSE || mode == MODE_FUSED) {
+        if (!make_map(&q, base + pl.qp, prow, 128, false) || !make_map(&kb, base + pl.kp, prow, g.b, false) ||
+            !make_map(&vb, base + pl.vp, prow, g.b, true))
             return cudaErrorInvalidValue;
-        const int q_tiles = pl.np_pad / 128;
-        return g.b == 128 ? launch_mode<MODE_SPARSE, 128>(prm, q, k0, v0, k0, v0, q_tiles, st)
-                          : launch_mode<MODE_SPARSE, 64>(prm, q, k0, v0, k0, v0, q_tiles, st);
+        if (mode == MODE_FUSED && has_sp) {
+            if (!make_map(&ka, base + pl.ks, srow, g.b, false) || !make_map(&va, base + pl.vs, srow, g.b, true))
+                return cudaErrorInvalidValue;
+        } else {
+            ka = kb;
+            va = vb;
+        }
+        prm.q_tiles = patch_tiles;
+        const int ctas = patch_tiles * g.H;
+        if (mode == MODE_SPARSE)
+            return g.b == 128 ? launch_mode<MODE_SPARSE, 128>(prm, q, ka, va, kb, vb, ctas, st)
+                              : launch_mode<MODE_SPARSE, 64>(prm, q, ka, va, kb, vb, ctas, st);
+        return g.b == 128 ? launch_mode<MODE_FUSED, 128>(prm, q, ka, va, kb, vb, ctas, st)
+                          : launch_mode<MODE_FUSED, 64>(prm, q, ka, va, kb, vb, ctas, st);
     }
-    if (g.Ns == 0) return cudaSuccess;
-    if (!make_map(&k0, base + pl.ks, srow, 128, false) || !make_map(&v0, base + pl.vs, srow, 128, true))
+    if (!has_sp) return cudaSuccess;
+    if (!make_map(&ka, base + pl.ks, srow, 128, false) || !make_map(&va, base + pl.vs, srow, 128, true))
         return cudaErrorInvalidValue;
     if (mode == MODE_PATCH_SPECIAL) {
         if (!make_map(&q, base + pl.qp, prow, 128, false)) return cudaErrorInvalidValue;
-        return launch_mode<MODE_PATCH_SPECIAL, 128>(prm, q, k0, v0, k0, v0, pl.np_pad / 128, st);
+        prm.q_tiles = patch_tiles;
+        return launch_mode<MODE_PATCH_SPECIAL, 128>(prm, q, ka, va, ka, va, patch_tiles * g.H, st);
     }
-    if (!make_map(&q, base + pl.qs, srow, 128, false) || !make_map(&k1, base + pl.kp, prow, 128, false) ||
-        !make_map(&v1, base + pl.vp, prow, 128, true))
+    if (!make_map(&q, base + pl.qs, srow, 128, false) || !make_map(&kb, base + pl.kp, prow, 128, false) ||
+        !make_map(&vb, base + pl.vp, prow, 128, true))
         return cudaErrorInvalidValue;
-    return launch_mode<MODE_SPECIAL_ALL, 128>(prm, q, k0, v0, k1, v1, pl.ns_pad / 128, st);
+    prm.q_tiles = pl.ns_pad / 128;
+    cudaError_t e = launch_mode<MODE_SPECIAL_ALL, 128>(prm, q, ka, va, kb, vb, prm.q_tiles * pl.nsplit * g.H, st);
+    if (e != cudaSuccess) return e;
+    special_combine_kernel<<<num_sms() * 4, 256, 0, st>>>(g, pl, prm.spart, prm.slse, prm.out);
+    return cudaGetLastError();
 }
 
 }  // namespace bsa

@@ -12,8 +12,11 @@ namespace bsa {
 struct PackedLayout {
     int np_pad;          // patch rows per head, multiple of 128
     int ns_pad;          // special rows per head, multiple of 128 (0 without specials)
+    int nsplit;          // key-range splits of the special-query attention
     size_t qp, kp, vp;   // byte offsets of the patch arrays   [H][np_pad][64]
     size_t qs, ks, vs;   // byte offsets of the special arrays [H][ns_pad][64]
+    size_t spart;        // fp32 [nsplit][H][ns_pad][64] partial outputs of special queries
+    size_t slse;         // fp32 [nsplit][H][ns_pad] their log-sum-exp values
     size_t bytes;        // total
 };
 
@@ -21,6 +24,9 @@ __host__ __device__ inline PackedLayout packed_layout(const Geo& g) {
     PackedLayout pl;
     pl.np_pad = (g.Np + 127) / 128 * 128;
     pl.ns_pad = (g.Ns + 127) / 128 * 128;
+    // special queries see every key: split the key range into chunks of about 64 tiles
+    const int n_all = pl.ns_pad / 128 + pl.np_pad / 128;
+    pl.nsplit = g.Ns == 0 ? 0 : (n_all + 63) / 64 > 16 ? 16 : (n_all + 63) / 64;
     const size_t patch = (size_t)g.H * pl.np_pad * 128;
     const size_t spec = (size_t)g.H * pl.ns_pad * 128;
     pl.qp = 0;
@@ -29,7 +35,9 @@ __host__ __device__ inline PackedLayout packed_layout(const Geo& g) {
     pl.qs = pl.vp + patch;
     pl.ks = pl.qs + spec;
     pl.vs = pl.ks + spec;
-    pl.bytes = pl.vs + spec;
+    pl.spart = pl.vs + spec;
+    pl.slse = pl.spart + (size_t)pl.nsplit * g.H * pl.ns_pad * 64 * 4;
+    pl.bytes = pl.slse + ((size_t)pl.nsplit * g.H * pl.ns_pad * 4 + 1023) / 1024 * 1024;
     return pl;
 }
 
