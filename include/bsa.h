@@ -197,6 +197,32 @@ BSA_API bsa_status bsa_block_sparse_attn_fused(const bsa_layout* layout, const v
                                                int32_t* status_dev, bsa_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
+ * Allocation-free attention (bf16). The pages have no counterpart: this entry point
+ * exists for callers that cannot allocate device memory -- code running under a host
+ * framework whose memory pool owns every device allocation, or latency-critical loops in
+ * which cudaMalloc/cudaFree are not allowed because they may synchronize the device.
+ * It does what bsa_pack_qkv + bsa_special_dense (o_ps = NULL) + bsa_block_sparse_attn_fused
+ * do (every row of out: the special rows dense, the patch rows over the special keys and
+ * the kept blocks), but keeps the packed copy and the partial results in one static
+ * device array of BSA_NOALLOC_SCRATCH_BYTES inside the library instead of a workspace.
+ * The array exists on every GPU that loads the library until the process exits.
+ *   - Layers whose packed data (bsa_workspace_size) exceed BSA_NOALLOC_SCRATCH_BYTES are
+ *     rejected with BSA_ERR_UNSUPPORTED before anything is launched.
+ *   - No memory is allocated or freed. The first call on a device looks up the device
+ *     address of the array (cudaGetSymbolAddress) with that device current; make that
+ *     first call before any stream capture.
+ *   - All calls share the array and it keeps the last call's contents; every byte a call
+ *     reads is written earlier by the same call, so nothing needs clearing. Calls that
+ *     overlap on the GPU (other streams, other threads) race on the array: serialize them.
+ *   q, k, v : device, [N, H, d] bf16;  kv_idx, kv_cnt : as written by bsa_predict_mask
+ *   out     : device, [N, H, d] bf16, every row written
+ */
+#define BSA_NOALLOC_SCRATCH_BYTES (64u << 20)
+BSA_API bsa_status bsa_attention_noalloc(const bsa_layout* layout, const void* q, const void* k,
+                                         const void* v, const uint16_t* kv_idx, const int32_t* kv_cnt,
+                                         void* out, int32_t* status_dev, bsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
  * Host helpers (no device work).
  */
 /* B = ceil(F P / b). */

@@ -41,6 +41,7 @@ _SIGS = {
     "bsa_special_dense": [_LP, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp, _i32p, _st],
     "bsa_merge": [_LP, _vp, _vp, _vp, _vp, _vp, _i32p, _st],
     "bsa_block_sparse_attn_fused": [_LP, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp, _i32p, _st],
+    "bsa_attention_noalloc": [_LP, _vp, _vp, _vp, _vp, _vp, _vp, _i32p, _st],
     "bsa_num_blocks": [_LP, ctypes.POINTER(ctypes.c_int32)],
     "bsa_workspace_size": [_LP, ctypes.POINTER(ctypes.c_size_t)],
     "bsa_k_from_rho": [ctypes.c_int32, ctypes.c_double, ctypes.POINTER(ctypes.c_int32)],
@@ -174,3 +175,9 @@ def bsa_block_sparse_attn_fused(layout, q, k, v, workspace, workspace_bytes, kv_
                                 stream=0) -> None:
     _check("bsa_block_sparse_attn_fused", load().bsa_block_sparse_attn_fused(
         ctypes.byref(layout), q, k, v, workspace, workspace_bytes, kv_idx, kv_cnt, out, status, stream))
+
+
+def bsa_attention_noalloc(layout, q, k, v, kv_idx, kv_cnt, out, status=0, stream=0) -> None:
+    """Steps 4-6 for bf16 layers with the library's static scratch (no workspace argument)."""
+    _check("bsa_attention_noalloc", load().bsa_attention_noalloc(
+        ctypes.byref(layout), q, k, v, kv_idx, kv_cnt, out, status, stream))

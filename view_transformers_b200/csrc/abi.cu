@@ -82,6 +82,10 @@ bsa_status check_ws(const Geo& g, const void* ws, size_t bytes) {
 }
 
 }  // namespace
+
+// Layout validation for entry points defined in other files.
+bsa_status make_geo_checked(const bsa_layout* L, Geo* g) { return make_geo(L, g); }
+
 }  // namespace bsa
 
 using namespace bsa;
