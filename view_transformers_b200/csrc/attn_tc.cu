@@ -351,9 +351,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             __syncwarp();
             if (lane == 0) mbar_arrive(&ctl.s_free);   // the next QK^T may overwrite S
             float mt = -INFINITY;
-            if (full) {
+            if (full) {   // 3-input max tree: short dependency chains
+                float acc[8];
 #pragma unroll
-                for (int c = 0; c < BKV; ++c) mt = fmaxf(mt, __uint_as_float(s[c]));
+                for (int i = 0; i < 8; ++i) acc[i] = __uint_as_float(s[i]);
+#pragma unroll
+                for (int c = 8; c < BKV; c += 2)
+                    acc[(c / 2) & 7] = max3f(acc[(c / 2) & 7], __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+                mt = max3f(max3f(acc[0], acc[1], acc[2]), max3f(acc[3], acc[4], acc[5]), fmaxf(acc[6], acc[7]));
             } else if (member) {
 #pragma unroll
                 for (int c = 0; c < BKV; ++c)
@@ -369,14 +374,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             // s[2i+1] were read
             float rs = 0.f;
             if (full) {
+                float r[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // independent partial sums
 #pragma unroll
                 for (int c = 0; c < BKV; c += 2) {
                     const float p0 = ex2_approx(fmaf(__uint_as_float(s[c]), kScaleLog2, -m_ref));
                     const float p1 = ex2_approx(fmaf(__uint_as_float(s[c + 1]), kScaleLog2, -m_ref));
-                    rs += p0 + p1;
+                    r[(c / 2) & 3] += p0;
+                    r[((c / 2) & 3) + 4] += p1;
                     const __half2 hp = __floats2half2_rn(p0, p1);
                     s[c / 2] = *reinterpret_cast<const uint32_t*>(&hp);
                 }
+                rs = ((r[0] + r[1]) + (r[2] + r[3])) + ((r[4] + r[5]) + (r[6] + r[7]));
             } else {
 #pragma unroll
                 for (int c = 0; c < BKV; c += 2) {
