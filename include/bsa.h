@@ -83,7 +83,9 @@ typedef struct {
  * pq[h, j, :] = mean of Q[row(p), h, :] over the patch tokens p of block j (the
  * divisor is the block's real token count); the same for pk from K.
  *   q, k    : device, [N, H, d] of layout->dtype
- *   pq, pk  : device, float32 [H, B, d]
+ *   pq      : device, float32 [H, B, d]
+ *   pk      : device, float32 [H, d, B] (dimension-major: the score pass of
+ *             bsa_predict_mask reads 32 consecutive blocks of one dimension per load)
  */
 BSA_API bsa_status bsa_pool_qk(const bsa_layout* layout, const void* q, const void* k,
                        float* pq, float* pk, int32_t* status_dev, bsa_stream_t stream);
@@ -97,7 +99,7 @@ BSA_API bsa_status bsa_pool_qk(const bsa_layout* layout, const void* q, const vo
  * k_h = floor(B (1 - rho) + 1e-9) for every head when head_density is NULL; otherwise
  * k_h = clamp(floor(B head_density[h] + 1e-9), 1, B) and rho only validates that
  * sum_h head_density[h] = H (1 - rho) within 1e-9 * H.
- *   pq, pk        : device, float32 [H, B, d] (from bsa_pool_qk)
+ *   pq, pk        : device, float32 [H, B, d] and [H, d, B] (from bsa_pool_qk)
  *   rho, tau      : in [0, 1]
  *   head_density  : host, double [H] in [0, 1], or NULL
  *   mask_bits     : device, uint32 [H, B, ceil(B/32)] (bit j%32 of word j/32 = block j

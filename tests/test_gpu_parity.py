@@ -58,7 +58,7 @@ def test_mask_and_layer(w):
     assert res["status"] == 0
     lay, PQ, PK, kh, om = _oracle_mask(w, x, res)
     # pooling
-    assert max_abs(res["pq"], PQ) < 1e-5 and max_abs(res["pk"], PK) < 1e-5
+    assert max_abs(res["pq"], PQ) < 1e-5 and max_abs(res["pk"], PK.transpose(0, 2, 1)) < 1e-5
     # mask
     rep = compare_mask(om, res["selected"], w.tau)
     print(f"{w.name}: mask rows {rep.rows} exact {rep.exact} exempt {rep.exempt} failed {rep.failed}")

@@ -4,14 +4,22 @@
 // n = min(B, max(k_h, n_tau)) blocks of the ranking (p descending, lower index first),
 // n_tau = smallest n with cumulative mass >= tau.
 //
-// One warp per query-block row, W rows (warps) of one head per CTA so that each PK tile
-// staged in shared memory serves W rows. The [H, B, B] score matrix is never written to
-// HBM. Instead of sorting a row, the selection is a radix select on the order-preserving
-// 32-bit image of the fp32 score:
+// One CTA holds R query-block rows of one head. The [H, B, B] score matrix is never
+// written to HBM: a CTA computes its R x B score rows into shared memory, then each warp
+// selects on one row at a time.
+//
+// Scores (FMA-bound): pooled K is stored dimension-major ([H][d][B]), so a warp reads 32
+// consecutive blocks of one dimension per load straight from L2; each lane accumulates
+// two blocks x R rows (2R independent FMA chains) with the R query values of a dimension
+// broadcast from shared memory, so one shared-memory wavefront feeds 8 FMAs per lane.
+//
+// Selection: instead of sorting a row, a radix select on the order-preserving 32-bit
+// image of the fp32 score:
 //   - the common leading bits of the row's keys are skipped (near-uniform rows share
 //     sign and exponent), then 8-bit digits are resolved from the top;
 //   - the CDF bound uses per-digit fp64 mass histograms (the target is tau * sum_j e_j,
-//     e_j = exp(s_ij - max_j s_ij), so no division is needed);
+//     e_j = exp(s_ij - max_j s_ij), so no division is needed); with tau = 0 no
+//     exponential is evaluated at all;
 //   - ties (equal keys) are taken in ascending block index.
 // The kept blocks are then emitted in ascending index order with warp ballots.
 #include <cfloat>
@@ -21,18 +29,31 @@
 namespace bsa {
 namespace {
 
-constexpr int kKeyTile = 64;      // PK rows staged per pass
-constexpr int kPkStride = 68;     // padded row (floats): conflict-free 16-byte loads
+constexpr int kMaxWarps = 16;
 constexpr int kRadix = 256;
+constexpr int kDim = 64;
+
+// Masses are fixed-point: e_j * 2^40 rounded to an integer. With at most 2^13 blocks every
+// partial sum is an integer below 2^53, so the sums are exact in any order (atomics stay
+// deterministic) and convert to double without rounding.
+constexpr float kFix = 1099511627776.0f;   // 2^40
 
 struct WarpHist {
     unsigned int cnt[kRadix];
-    double mass[kRadix];
+    unsigned long long mass[kRadix];
 };
 
 __device__ __forceinline__ uint32_t order_key(float s) {
     const uint32_t u = __float_as_uint(s);
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float key_value(uint32_t u) {
+    return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
+
+__device__ __forceinline__ unsigned long long fix_mass(float s, float mx) {
+    return __float2ull_rn(expf(s - mx) * kFix);
 }
 
 __device__ __forceinline__ unsigned lanemask_lt() {
@@ -41,22 +62,102 @@ __device__ __forceinline__ unsigned lanemask_lt() {
     return m;
 }
 
-// Result of a descending radix select over a row's keys.
+// Equal-width score buckets over [lo, max]: digit(s) = min(255, floor((s - lo) * scale)) is
+// monotone in s, so a higher bucket holds strictly larger scores and equal scores share a
+// bucket. sel >= 0 restricts a pass to the members of one bucket.
+struct Bucket {
+    float lo, scale;
+    int sel;
+    __device__ __forceinline__ int digit(float s) const {
+        return min(kRadix - 1, __float2int_rz((s - lo) * scale));
+    }
+    __device__ __forceinline__ bool member(float s) const { return sel < 0 || digit(s) == sel; }
+};
+
+// Result of a descending selection over a row.
 struct Cut {
     uint32_t t;        // threshold key
     int greater;       // elements with key > t
     int take;          // elements with key == t that are kept (lowest indices first)
 };
 
-// Finds the cut for either the n largest keys (mass_mode = false, target_n) or the smallest
-// prefix of the ranking whose mass reaches target_m (mass_mode = true). Warp-collective.
-__device__ Cut radix_cut(const uint32_t* keys, const float* e, int B, bool mass_mode, int target_n,
-                         double target_m, WarpHist* hist, int lane) {
-    // common prefix of all keys
+// One digit of a descending select: the digit where the running count reaches rem_n
+// (mass_mode = false) or the running mass reaches rem_m, with what lies above it.
+struct Pick {
+    int digit;
+    unsigned above_c, at_c;
+    double above_m;
+};
+
+__device__ Pick scan_hist(const WarpHist* hist, bool mass_mode, int rem_n, double rem_m, int lane) {
+    // lane l owns digits 255-8l .. 248-8l (descending); exclusive scan in lane order
+    unsigned c[8];
+    double m[8];
+    unsigned lc = 0;
+    double lm = 0.0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const int dg = kRadix - 1 - (8 * lane + q);
+        c[q] = hist->cnt[dg];
+        m[q] = mass_mode ? (double)hist->mass[dg] : 0.0;
+        lc += c[q];
+        lm += m[q];
+    }
+    unsigned ic = lc;
+    double im = lm;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned oc = __shfl_up_sync(0xffffffffu, ic, o);
+        const double om = mass_mode ? __shfl_up_sync(0xffffffffu, im, o) : 0.0;
+        if (lane >= o) { ic += oc; im += om; }
+    }
+    const unsigned ec = ic - lc;
+    const double em = im - lm;     // exact: integers below 2^53
+    const bool hit = lc > 0 && (mass_mode ? (em < rem_m && rem_m <= im)
+                                          : (ec < (unsigned)rem_n && (unsigned)rem_n <= ic));
+    const unsigned hits = __ballot_sync(0xffffffffu, hit);
+    // no lane reaches the target: cut at the lowest non-empty digit (keeps every candidate)
+    const int src = hits ? __ffs(hits) - 1 : 31 - __clz(__ballot_sync(0xffffffffu, lc > 0));
+    Pick pk{0, 0u, 0u, 0.0};
+    if (lane == src) {
+        unsigned accc = ec;
+        double accm = em;
+        int qsel = -1;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const bool here = hits ? (qsel < 0 && (mass_mode ? (accm + m[q] >= rem_m)
+                                                            : (accc + c[q] >= (unsigned)rem_n)))
+                                   : c[q] > 0;   // fallback: the last non-empty digit wins
+            if (here) {
+                qsel = q;
+                pk.above_c = accc;
+                pk.above_m = accm;
+                pk.at_c = c[q];
+            }
+            if (qsel < 0 || !hits) { accc += c[q]; accm += m[q]; }
+        }
+        pk.digit = kRadix - 1 - (8 * lane + qsel);
+    }
+    pk.digit = __shfl_sync(0xffffffffu, pk.digit, src);
+    pk.above_c = __shfl_sync(0xffffffffu, pk.above_c, src);
+    pk.at_c = __shfl_sync(0xffffffffu, pk.at_c, src);
+    if (mass_mode) pk.above_m = __shfl_sync(0xffffffffu, pk.above_m, src);
+    return pk;
+}
+
+// Radix select over the order-preserving keys of the candidates (members of f, ncand of
+// them), below `greater` elements already kept: the cut for rem_n more elements
+// (mass_mode = false) or for rem_m more mass. Warp-collective.
+__device__ Cut radix_cut(const float* s, int B, float mx, Bucket f, int ncand, bool mass_mode,
+                         int greater, int rem_n, double rem_m, WarpHist* hist, int lane) {
     uint32_t kmin = 0xffffffffu, kmax = 0u;
     for (int j = lane; j < B; j += 32) {
-        kmin = min(kmin, keys[j]);
-        kmax = max(kmax, keys[j]);
+        const float sj = s[j];
+        if (f.member(sj)) {
+            const uint32_t u = order_key(sj);
+            kmin = min(kmin, u);
+            kmax = max(kmax, u);
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -67,109 +168,47 @@ __device__ Cut radix_cut(const uint32_t* keys, const float* e, int B, bool mass_
     int hb = diff ? 31 - __clz(diff) : -1;      // highest differing bit
     uint32_t fixed_mask = hb >= 31 ? 0u : (0xffffffffu << (hb + 1));
     uint32_t prefix = kmax & fixed_mask;
-    int greater = 0;
-    int rem_n = target_n;
-    double rem_m = target_m;
+    int ties = ncand;                            // all candidates equal when no digit is resolved
 
     while (hb >= 0) {
-        if (mass_mode && rem_m <= 0.0) {   // rounding left no mass to cover: keep one more
+        if (mass_mode && rem_m <= 0.0) {   // nothing left to cover: keep one more
             mass_mode = false;
             rem_n = 1;
         }
         const int width = hb + 1 >= 8 ? 8 : hb + 1;
         const int shift = hb + 1 - width;
         const uint32_t dmask = (1u << width) - 1u;
+        __syncwarp();
         for (int x = lane; x < kRadix; x += 32) {
             hist->cnt[x] = 0u;
-            hist->mass[x] = 0.0;
+            if (mass_mode) hist->mass[x] = 0ull;
         }
         __syncwarp();
         for (int j = lane; j < B; j += 32) {
-            const uint32_t u = keys[j];
-            if ((u & fixed_mask) == prefix) {
+            const float sj = s[j];
+            const uint32_t u = order_key(sj);
+            if ((u & fixed_mask) == prefix && f.member(sj)) {
                 const int dg = (u >> shift) & dmask;
                 atomicAdd(&hist->cnt[dg], 1u);
-                if (mass_mode) atomicAdd(&hist->mass[dg], (double)e[j]);
+                if (mass_mode) atomicAdd(&hist->mass[dg], fix_mass(sj, mx));
             }
         }
         __syncwarp();
-        // lane l owns digits 255-8l .. 248-8l (descending); exclusive scan in lane order
-        unsigned c[8];
-        double m[8];
-        unsigned lc = 0;
-        double lm = 0.0;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const int dg = kRadix - 1 - (8 * lane + q);
-            c[q] = hist->cnt[dg];
-            m[q] = mass_mode ? hist->mass[dg] : 0.0;
-            lc += c[q];
-            lm += m[q];
-        }
-        unsigned ic = lc;
-        double im = lm;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const unsigned oc = __shfl_up_sync(0xffffffffu, ic, o);
-            const double om = __shfl_up_sync(0xffffffffu, im, o);
-            if (lane >= o) { ic += oc; im += om; }
-        }
-        unsigned ec = __shfl_up_sync(0xffffffffu, ic, 1);
-        double em = __shfl_up_sync(0xffffffffu, im, 1);
-        if (lane == 0) { ec = 0u; em = 0.0; }
-        const bool hit = lc > 0 && (mass_mode ? (em < rem_m && rem_m <= im)
-                                              : (ec < (unsigned)rem_n && (unsigned)rem_n <= ic));
-        const unsigned hits = __ballot_sync(0xffffffffu, hit);
-        // no lane reaches the target (mass above the histogram total by rounding): cut at
-        // the lowest non-empty digit, which keeps every candidate.
-        const int src = hits ? __ffs(hits) - 1 : 31 - __clz(__ballot_sync(0xffffffffu, lc > 0));
-        int dsel = 0;
-        unsigned above_c = 0;
-        double above_m = 0.0;
-        if (lane == src) {
-            int qsel = -1;
-            if (hits) {
-                unsigned accc = ec;
-                double accm = em;
-                for (int q = 0; q < 8 && qsel < 0; ++q) {
-                    if (mass_mode ? (accm + m[q] >= rem_m) : (accc + c[q] >= (unsigned)rem_n)) qsel = q;
-                    else { accc += c[q]; accm += m[q]; }
-                }
-            }
-            if (qsel < 0)
-                for (int q = 0; q < 8; ++q) if (c[q] > 0) qsel = q;   // lowest non-empty digit
-            above_c = ec;
-            above_m = em;
-            for (int q = 0; q < qsel; ++q) { above_c += c[q]; above_m += m[q]; }
-            dsel = kRadix - 1 - (8 * lane + qsel);
-        }
-        dsel = __shfl_sync(0xffffffffu, dsel, src);
-        above_c = __shfl_sync(0xffffffffu, above_c, src);
-        above_m = __shfl_sync(0xffffffffu, above_m, src);
-        greater += (int)above_c;
-        rem_n -= (int)above_c;
-        rem_m -= above_m;
-        prefix |= ((uint32_t)dsel) << shift;
+        const Pick pk = scan_hist(hist, mass_mode, rem_n, rem_m, lane);
+        greater += (int)pk.above_c;
+        rem_n -= (int)pk.above_c;
+        rem_m -= pk.above_m;
+        prefix |= ((uint32_t)pk.digit) << shift;
         fixed_mask |= dmask << shift;
+        ties = (int)pk.at_c;        // after the last digit: the candidates equal to prefix
         hb = shift - 1;
-        __syncwarp();
-    }
-    // every key equal to `prefix` is now a tie at the cut
-    int ties = 0;
-    float et = 0.f;
-    for (int j = lane; j < B; j += 32) {
-        if (keys[j] == prefix) { ++ties; et = e[j]; }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        ties += __shfl_xor_sync(0xffffffffu, ties, o);
-        et = fmaxf(et, __shfl_xor_sync(0xffffffffu, et, o));
     }
     Cut cut;
     cut.t = prefix;
     cut.greater = greater;
     if (mass_mode) {
-        int need = rem_m <= 0.0 ? 1 : (int)ceil(rem_m / (double)et);
+        const double et = (double)fix_mass(key_value(prefix), mx);
+        const int need = rem_m <= 0.0 ? 1 : et > 0.0 ? (int)ceil(rem_m / et) : ties;
         cut.take = max(1, min(ties, need));
     } else {
         cut.take = max(0, min(ties, rem_n));
@@ -177,91 +216,123 @@ __device__ Cut radix_cut(const uint32_t* keys, const float* e, int B, bool mass_
     return cut;
 }
 
-__global__ void mask_kernel(Geo g, MaskParams mp, const float* __restrict__ pq,
-                            const float* __restrict__ pk, uint32_t* __restrict__ mask_bits,
-                            uint16_t* __restrict__ kv_idx, int32_t* __restrict__ kv_cnt,
-                            int32_t* status) {
-    extern __shared__ __align__(16) unsigned char smem[];
-    const int W = blockDim.x / 32;
-    const int warp = threadIdx.x / 32;
-    const int lane = threadIdx.x % 32;
-    const int h = blockIdx.y;
-    const int B = g.B;
-    const int i = blockIdx.x * W + warp;           // query block of this warp
-    const bool row_ok = i < B;
-
-    float* pk_tile = reinterpret_cast<float*>(smem);                    // [kKeyTile][kPkStride]
-    float* pq_rows = pk_tile + kKeyTile * kPkStride;                      // [W][64]
-    WarpHist* hists = reinterpret_cast<WarpHist*>(pq_rows + W * 64);      // [W]
-    unsigned char* rowbuf = reinterpret_cast<unsigned char*>(hists + W);  // [W][B] keys, [W][B] e
-    uint32_t* keys = reinterpret_cast<uint32_t*>(rowbuf) + (size_t)warp * B;
-    float* ex = reinterpret_cast<float*>(rowbuf + (size_t)W * B * 4) + (size_t)warp * B;
-    float* sc = ex;   // scores are kept in the e buffer until the softmax pass
-
-    const float* pk_h = pk + (size_t)h * B * 64;
-    for (int x = lane; x < 64; x += 32) pq_rows[warp * 64 + x] = row_ok ? pq[((size_t)h * B + i) * 64 + x] : 0.f;
-    const float scale = 0.125f;   // 1 / sqrt(64)
-
-    // ---- pooled scores, one 64-row PK tile at a time
-    for (int j0 = 0; j0 < B; j0 += kKeyTile) {
-        __syncthreads();
-        const int nrows = min(kKeyTile, B - j0);
-        for (int x = threadIdx.x; x < nrows * 16; x += blockDim.x) {
-            const int r = x / 16, c4 = x % 16;
-            const float4 v = __ldg(reinterpret_cast<const float4*>(pk_h + (size_t)(j0 + r) * 64) + c4);
-            *reinterpret_cast<float4*>(pk_tile + r * kPkStride + c4 * 4) = v;
-        }
-        __syncthreads();
-        if (row_ok) {
-            const float4* qv = reinterpret_cast<const float4*>(pq_rows + warp * 64);
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const int r = lane + 32 * half;
-                if (r < nrows) {
-                    const float4* kv = reinterpret_cast<const float4*>(pk_tile + r * kPkStride);
-                    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-#pragma unroll
-                    for (int c4 = 0; c4 < 16; ++c4) {
-                        const float4 qa = qv[c4];
-                        const float4 ka = kv[c4];
-                        a0 = fmaf(qa.x, ka.x, a0);
-                        a1 = fmaf(qa.y, ka.y, a1);
-                        a2 = fmaf(qa.z, ka.z, a2);
-                        a3 = fmaf(qa.w, ka.w, a3);
-                    }
-                    sc[j0 + r] = ((a0 + a1) + (a2 + a3)) * scale;
-                }
-            }
-        }
-    }
-    if (!row_ok) return;
+// The cut inside one bucket of at most 32 members: each lane takes one member and ranks it
+// against the others (score descending, index ascending).
+__device__ Cut small_cut(const float* s, int B, float mx, Bucket f, int m, bool mass_mode,
+                         int greater, int rem_n, double rem_m, WarpHist* hist, int lane) {
+    float* ls = reinterpret_cast<float*>(hist->cnt);      // [32] member scores
+    int* lj = reinterpret_cast<int*>(hist->cnt) + 32;     // [32] member indices
     __syncwarp();
+    int base = 0;
+    for (int j0 = 0; j0 < B; j0 += 32) {
+        const int j = j0 + lane;
+        const float sj = j < B ? s[j] : 0.f;
+        const bool pred = j < B && f.digit(sj) == f.sel;
+        const unsigned bal = __ballot_sync(0xffffffffu, pred);
+        const int pos = base + __popc(bal & lanemask_lt());
+        if (pred && pos < 32) { ls[pos] = sj; lj[pos] = j; }
+        base += __popc(bal);
+    }
+    __syncwarp();
+    const bool mine = lane < m;
+    const float cs = mine ? ls[lane] : -FLT_MAX;
+    const int cj = mine ? lj[lane] : 0x7fffffff;
+    const unsigned long long ce = (mass_mode && mine) ? fix_mass(cs, mx) : 0ull;
+    int rank = 0;
+    unsigned long long before = 0ull;
+    for (int t = 0; t < m; ++t) {
+        const float st = __shfl_sync(0xffffffffu, cs, t);
+        const int jt = __shfl_sync(0xffffffffu, cj, t);
+        const unsigned long long et = mass_mode ? __shfl_sync(0xffffffffu, ce, t) : 0ull;
+        if (st > cs || (st == cs && jt < cj)) { ++rank; before += et; }
+    }
+    const bool sel = mine && (mass_mode ? (double)before < rem_m : rank < rem_n);
+    const int nsel = __popc(__ballot_sync(0xffffffffu, sel));
+    // the last kept member (rank nsel - 1), or the first member when none is kept
+    const unsigned lastb = __ballot_sync(0xffffffffu, mine && rank == (nsel > 0 ? nsel - 1 : 0));
+    const uint32_t kt = order_key(__shfl_sync(0xffffffffu, cs, __ffs(lastb) - 1));
+    const int take = __popc(__ballot_sync(0xffffffffu, sel && order_key(cs) == kt));
+    Cut cut;
+    cut.t = kt;
+    cut.greater = greater + nsel - take;
+    cut.take = take;
+    return cut;
+}
 
-    // ---- softmax pieces: row max, e_j = exp(s_j - max), fp64 total
-    float mx = -FLT_MAX;
-    for (int j = lane; j < B; j += 32) mx = fmaxf(mx, sc[j]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    double tot = 0.0;
+// Selection and emission for one row (h, i) whose scores are s[0, B).
+__device__ void select_row(const float* s, int B, int h, int i, int k, double tau,
+                           WarpHist* hist, uint32_t* __restrict__ mask_bits,
+                           uint16_t* __restrict__ kv_idx, int32_t* __restrict__ kv_cnt,
+                           int32_t* status, int lane) {
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
     for (int j = lane; j < B; j += 32) {
-        const float s = sc[j];
-        keys[j] = order_key(s);
-        const float e = expf(s - mx);
-        ex[j] = e;
-        tot += (double)e;
+        const uint32_t u = order_key(s[j]);
+        kmin = min(kmin, u);
+        kmax = max(kmax, u);
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
-    __syncwarp();
+    for (int o = 16; o > 0; o >>= 1) {
+        kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+        kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+    }
+    const float mx = key_value(kmax);
+    const float smin = key_value(kmin);
+    const float scale = (float)kRadix / (mx - smin);
+    // equal-width buckets unless the range is zero (all equal, or only +0 / -0) or too
+    // narrow for a finite scale; the radix select then works on the key bits directly
+    const bool bucketed = kmin != kmax && isfinite(scale);
+    const Bucket all{smin, scale, -1};
 
-    // ---- dual threshold
-    const int k = mp.k[h];
-    WarpHist* hist = hists + warp;
+    // The cut for the first n_target elements (mass_mode = false) or for mass tau * T,
+    // T = sum_j e_j (mass_mode = true).
+    auto find_cut = [&](bool mass_mode, int n_target) -> Cut {
+        if (!bucketed) {
+            double rem_m = 0.0;
+            if (mass_mode) {
+                unsigned long long tot = 0ull;
+                for (int j = lane; j < B; j += 32) tot += fix_mass(s[j], mx);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+                rem_m = tau * (double)tot;
+            }
+            return radix_cut(s, B, mx, all, B, mass_mode, 0, n_target, rem_m, hist, lane);
+        }
+        __syncwarp();
+        for (int x = lane; x < kRadix; x += 32) {
+            hist->cnt[x] = 0u;
+            if (mass_mode) hist->mass[x] = 0ull;
+        }
+        __syncwarp();
+        for (int j = lane; j < B; j += 32) {
+            const float sj = s[j];
+            const int dg = all.digit(sj);
+            atomicAdd(&hist->cnt[dg], 1u);
+            if (mass_mode) atomicAdd(&hist->mass[dg], fix_mass(sj, mx));
+        }
+        __syncwarp();
+        double rem_m = 0.0;
+        if (mass_mode) {
+            unsigned long long tot = 0ull;
+            for (int x = lane; x < kRadix; x += 32) tot += hist->mass[x];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+            rem_m = tau * (double)tot;
+        }
+        const Pick pk = scan_hist(hist, mass_mode, n_target, rem_m, lane);
+        const Bucket f{smin, scale, pk.digit};
+        const int greater = (int)pk.above_c;
+        const int rem_n = n_target - (int)pk.above_c;
+        rem_m -= pk.above_m;
+        if (pk.at_c <= 32)
+            return small_cut(s, B, mx, f, (int)pk.at_c, mass_mode, greater, rem_n, rem_m, hist, lane);
+        return radix_cut(s, B, mx, f, (int)pk.at_c, mass_mode, greater, rem_n, rem_m, hist, lane);
+    };
+
     int n;
     Cut cut;
     bool have_cut = false;
-    if (mp.tau > 0.0) {
-        cut = radix_cut(keys, ex, B, true, 0, mp.tau * tot, hist, lane);
+    if (tau > 0.0) {
+        cut = find_cut(true, 0);
         const int n_tau = cut.greater + cut.take;
         if (n_tau >= k) {
             n = n_tau;
@@ -277,7 +348,7 @@ __global__ void mask_kernel(Geo g, MaskParams mp, const float* __restrict__ pq,
         if (n <= 0) {
             cut.t = 0xffffffffu; cut.greater = 0; cut.take = 0;    // nothing above or at the cut
         } else {
-            cut = radix_cut(keys, ex, B, false, n, 0.0, hist, lane);
+            cut = find_cut(false, n);
         }
     }
     const bool none = n <= 0;
@@ -289,7 +360,7 @@ __global__ void mask_kernel(Geo g, MaskParams mp, const float* __restrict__ pq,
     for (int j0 = 0; j0 < B; j0 += 32) {
         const int j = j0 + lane;
         const bool valid = j < B;
-        const uint32_t u = valid ? keys[j] : 0u;
+        const uint32_t u = valid ? order_key(s[j]) : 0u;
         const bool tie = valid && !none && u == cut.t;
         const unsigned tb = __ballot_sync(0xffffffffu, tie);
         const int trank = taken_ties + __popc(tb & lanemask_lt());
@@ -306,23 +377,138 @@ __global__ void mask_kernel(Geo g, MaskParams mp, const float* __restrict__ pq,
     }
 }
 
+// R query-block rows i0 .. i0+R-1 of head h per CTA.
+template <int R>
+__global__ void __launch_bounds__(32 * kMaxWarps)
+mask_kernel(Geo g, MaskParams mp, const float* __restrict__ pq, const float* __restrict__ pk,
+            uint32_t* __restrict__ mask_bits, uint16_t* __restrict__ kv_idx,
+            int32_t* __restrict__ kv_cnt, int32_t* status) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int W = blockDim.x / 32;
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    const int h = blockIdx.y;
+    const int B = g.B;
+    const int i0 = blockIdx.x * R;
+
+    float* qT = reinterpret_cast<float*>(smem);                        // [d][R]
+    WarpHist* hists = reinterpret_cast<WarpHist*>(qT + kDim * R);      // [W]
+    float* sc = reinterpret_cast<float*>(hists + W);                   // [R][B]
+
+    for (int x = threadIdx.x; x < R * kDim; x += blockDim.x) {
+        const int r = x / kDim, d = x % kDim;
+        qT[d * R + r] = i0 + r < B ? pq[((size_t)h * B + i0 + r) * kDim + d] : 0.f;
+    }
+    __syncthreads();
+
+    // ---- pooled scores: 64-block chunks round-robin over the warps
+    const float* pk_h = pk + (size_t)h * kDim * B;
+    const float scale = 0.125f;   // 1 / sqrt(64)
+    const int nchunk = (B + 63) / 64;
+    for (int c = warp; c < nchunk; c += W) {
+        const int j0 = c * 64 + lane;
+        const int j1 = j0 + 32;
+        const bool v0 = j0 < B, v1 = j1 < B;
+        const float* p0 = pk_h + (v0 ? j0 : 0);
+        const float* p1 = pk_h + (v1 ? j1 : 0);
+        float a0[R], a1[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) { a0[r] = 0.f; a1[r] = 0.f; }
+        float k0[8], k1[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            k0[u] = __ldg(p0 + (size_t)u * B);
+            k1[u] = __ldg(p1 + (size_t)u * B);
+        }
+#pragma unroll 1
+        for (int d0 = 0; d0 < kDim; d0 += 8) {
+            float n0[8], n1[8];
+            if (d0 + 8 < kDim) {   // next eight dimensions in flight during this group's FMAs
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    n0[u] = __ldg(p0 + (size_t)(d0 + 8 + u) * B);
+                    n1[u] = __ldg(p1 + (size_t)(d0 + 8 + u) * B);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const float* qd = qT + (d0 + u) * R;
+#pragma unroll
+                for (int r4 = 0; r4 < R; r4 += (R >= 4 ? 4 : R)) {
+                    float qv[4];
+                    if constexpr (R >= 4) {
+                        const float4 t = *reinterpret_cast<const float4*>(qd + r4);
+                        qv[0] = t.x; qv[1] = t.y; qv[2] = t.z; qv[3] = t.w;
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < R; ++e) qv[e] = qd[e];
+                    }
+#pragma unroll
+                    for (int e = 0; e < (R >= 4 ? 4 : R); ++e) {
+                        a0[r4 + e] = fmaf(qv[e], k0[u], a0[r4 + e]);
+                        a1[r4 + e] = fmaf(qv[e], k1[u], a1[r4 + e]);
+                    }
+                }
+            }
+            if (d0 + 8 < kDim) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) { k0[u] = n0[u]; k1[u] = n1[u]; }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            if (v0) sc[(size_t)r * B + j0] = a0[r] * scale;
+            if (v1) sc[(size_t)r * B + j1] = a1[r] * scale;
+        }
+    }
+    __syncthreads();
+
+    // ---- selection: warp w takes rows w, w + W, ...
+    for (int r = warp; r < R; r += W) {
+        const int i = i0 + r;
+        if (i >= B) break;
+        select_row(sc + (size_t)r * B, B, h, i, mp.k[h], mp.tau, hists + warp, mask_bits, kv_idx,
+                   kv_cnt, status, lane);
+    }
+}
+
+template <int R>
+size_t mask_smem(int B, int W) {
+    return (size_t)kDim * R * 4 + sizeof(WarpHist) * W + (size_t)R * B * 4;
+}
+
+template <int R>
+cudaError_t launch_rows(const Geo& g, int W, const MaskParams& mp, const float* pq, const float* pk,
+                        uint32_t* mask_bits, uint16_t* kv_idx, int32_t* kv_cnt, int32_t* status,
+                        cudaStream_t st) {
+    const size_t smem = mask_smem<R>(g.B, W);
+    cudaError_t e = cudaFuncSetAttribute(mask_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((g.B + R - 1) / R, g.H);
+    mask_kernel<R><<<grid, 32 * W, smem, st>>>(g, mp, pq, pk, mask_bits, kv_idx, kv_cnt, status);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_mask(const Geo& g, const MaskParams& mp, const float* pq, const float* pk,
                         uint32_t* mask_bits, uint16_t* kv_idx, int32_t* kv_cnt,
                         int32_t* status, cudaStream_t st) {
-    const size_t fixed = (size_t)kKeyTile * kPkStride * 4;
-    const size_t per_warp = 64 * 4 + sizeof(WarpHist) + (size_t)g.B * 8;
-    const size_t budget = 200 * 1024;
-    int W = (int)((budget - fixed) / per_warp);
-    W = W > 8 ? 8 : W;
-    if (W < 1) return cudaErrorInvalidValue;
-    const size_t smem = fixed + W * per_warp;
-    cudaError_t e = cudaFuncSetAttribute(mask_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    const dim3 grid((g.B + W - 1) / W, g.H);
-    mask_kernel<<<grid, 32 * W, smem, st>>>(g, mp, pq, pk, mask_bits, kv_idx, kv_cnt, status);
-    return cudaGetLastError();
+    // 16 warps: the selection is a chain of dependent warp-wide steps per row, so it runs
+    // best with one row per warp and many rows in flight
+    const int W = kMaxWarps;
+    // the most rows per CTA whose score rows fit in shared memory
+    const size_t limit = 227 * 1024;
+    if (mask_smem<16>(g.B, W) <= limit)
+        return launch_rows<16>(g, W, mp, pq, pk, mask_bits, kv_idx, kv_cnt, status, st);
+    if (mask_smem<8>(g.B, W) <= limit)
+        return launch_rows<8>(g, W, mp, pq, pk, mask_bits, kv_idx, kv_cnt, status, st);
+    if (mask_smem<4>(g.B, W) <= limit)
+        return launch_rows<4>(g, W, mp, pq, pk, mask_bits, kv_idx, kv_cnt, status, st);
+    if (mask_smem<1>(g.B, W) <= limit)
+        return launch_rows<1>(g, W, mp, pq, pk, mask_bits, kv_idx, kv_cnt, status, st);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace bsa

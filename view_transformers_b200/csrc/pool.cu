@@ -3,7 +3,8 @@
 // patch tokens of the concatenated patch sequence, per head, accumulated in fp32.
 //
 // HBM-bound: every patch row of Q and K is read once (Np * H * d elements each), the
-// pooled [H, B, d] fp32 tensors are written once. One CTA per (block, Q|K); each warp
+// pooled fp32 tensors are written once: pq as [H, B, d], pk dimension-major as [H, d, B]
+// (the layout the score pass of the mask kernel reads with coalesced loads). One CTA per (block, Q|K); each warp
 // reads whole 16-byte chunks of consecutive rows (a row holds all heads, 2 KB in bf16
 // at H = 16), so every load is a coalesced 512-byte warp transaction. Row groups inside
 // the CTA keep 8-16 independent 16-byte loads in flight per thread.
@@ -68,7 +69,9 @@ pool_kernel(Geo g, const T* __restrict__ q, const T* __restrict__ k, float* __re
             const int el = c0 * V + e;
             const int h = el / g.d;
             const int dd = el - h * g.d;
-            dst[((size_t)h * g.B + j) * g.d + dd] = s / count;
+            const size_t at = blockIdx.y == 0 ? ((size_t)h * g.B + j) * g.d + dd     // pq [H][B][d]
+                                              : ((size_t)h * g.d + dd) * g.B + j;    // pk [H][d][B]
+            dst[at] = s / count;
         }
         __syncthreads();
     }

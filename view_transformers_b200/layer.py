@@ -49,7 +49,7 @@ class BlockSparseLayer:
         words = (B + 31) // 32
         self.buf = Buffers(
             pq=torch.empty((H, B, d), dtype=torch.float32, device=dev),
-            pk=torch.empty((H, B, d), dtype=torch.float32, device=dev),
+            pk=torch.empty((H, d, B), dtype=torch.float32, device=dev),   # dimension-major
             mask_bits=torch.empty((H, B, words), dtype=torch.int32, device=dev),
             kv_idx=torch.empty((H, B, B), dtype=torch.int16, device=dev),
             kv_cnt=torch.empty((H, B), dtype=torch.int32, device=dev),
