@@ -13,15 +13,18 @@
 // two blocks x R rows (2R independent FMA chains) with the R query values of a dimension
 // broadcast from shared memory, so one shared-memory wavefront feeds 8 FMAs per lane.
 //
-// Selection: instead of sorting a row, a radix select on the order-preserving 32-bit
-// image of the fp32 score:
-//   - the common leading bits of the row's keys are skipped (near-uniform rows share
-//     sign and exponent), then 8-bit digits are resolved from the top;
-//   - the CDF bound uses per-digit fp64 mass histograms (the target is tau * sum_j e_j,
-//     e_j = exp(s_ij - max_j s_ij), so no division is needed); with tau = 0 no
-//     exponential is evaluated at all;
-//   - ties (equal keys) are taken in ascending block index.
-// The kept blocks are then emitted in ascending index order with warp ballots.
+// Selection: instead of sorting a row, a select over the fp32 scores in three steps:
+//   - one pass counts the row into 256 equal-width score buckets over [min, max] (with
+//     tau > 0 also their masses e_j = exp(s_ij - max_j s_ij)); the bucket where the
+//     running count reaches k, or the running mass reaches tau * sum_j e_j, holds the cut
+//     (the CDF bound needs no division);
+//   - a bucket of at most 32 members is finished by ranking its members against each other
+//     in one warp; a larger one by a radix select on the order-preserving 32-bit image of
+//     the scores of its members (common leading bits skipped, then 8-bit digits);
+//   - ties (equal scores) are taken in ascending block index.
+// Masses are summed as fixed-point integers, so every sum is exact and independent of the
+// order in which shared-memory atomics land. The kept blocks are then emitted in ascending
+// index order with warp ballots.
 #include <cfloat>
 
 #include "common.cuh"
