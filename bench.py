@@ -134,6 +134,7 @@ def stage_bytes(w) -> dict:
     return {
         "pool": 2 * w.n_patch * row * e + pooled,
         "pack": 3 * w.n_tokens * row * e + 3 * w.n_tokens * row * 2,
+        "pack_pool": 3 * w.n_tokens * row * e + 3 * w.n_tokens * row * 2 + pooled,
         "merge": 2 * w.n_patch * row * 4 + 2 * w.heads * w.n_patch * 4 + w.n_patch * row * e,
     }
 
@@ -147,13 +148,21 @@ def step_calls(L, q, k, v, path: str):
     status = b.status.data_ptr()
     lay = L.layout
     qp, kp, vp = q.data_ptr(), k.data_ptr(), v.data_ptr()
-    calls = [
-        ("pool", lambda: _lib.bsa_pool_qk(lay, qp, kp, b.pq.data_ptr(), b.pk.data_ptr(), status, sp), 1),
-        ("mask", lambda: _lib.bsa_predict_mask(lay, b.pq.data_ptr(), b.pk.data_ptr(), L.rho, L.tau, L.head_density,
-                                               b.mask_bits.data_ptr(), b.kv_idx.data_ptr(), b.kv_cnt.data_ptr(),
-                                               status, sp), 1),
-        ("pack", lambda: _lib.bsa_pack_qkv(lay, qp, kp, vp, L.ws_ptr, L.ws_bytes, status, sp), 1),
-    ]
+    mask = ("mask", lambda: _lib.bsa_predict_mask(lay, b.pq.data_ptr(), b.pk.data_ptr(), L.rho, L.tau,
+                                                  L.head_density, b.mask_bits.data_ptr(), b.kv_idx.data_ptr(),
+                                                  b.kv_cnt.data_ptr(), status, sp), 1)
+    if path == "fused":
+        calls = [
+            ("pack_pool", lambda: _lib.bsa_pack_pool_qkv(lay, qp, kp, vp, L.ws_ptr, L.ws_bytes, b.pq.data_ptr(),
+                                                         b.pk.data_ptr(), status, sp), 1),
+            mask,
+        ]
+    else:
+        calls = [
+            ("pool", lambda: _lib.bsa_pool_qk(lay, qp, kp, b.pq.data_ptr(), b.pk.data_ptr(), status, sp), 1),
+            mask,
+            ("pack", lambda: _lib.bsa_pack_qkv(lay, qp, kp, vp, L.ws_ptr, L.ws_bytes, status, sp), 1),
+        ]
     if path == "fused":
         calls += [
             ("special", lambda: _lib.bsa_special_dense(lay, qp, kp, vp, L.ws_ptr, L.ws_bytes, b.out.data_ptr(),
@@ -403,7 +412,8 @@ def main():
         "dense_ms_per_layer": dense_ms, "speedup_vs_dense": dense_ms / ms_per_step if dense_ms else None,
         "density": density_real, "sparsity": 1 - density_real,
         "stage_ms": stage_ms, "dense_stage_ms": {k_: float(np.mean(vs)) for k_, vs in dense_stage.items()},
-        "mask_prediction_gbs": sb["pool"] / ((stage_ms["pool"] + stage_ms["mask"]) * 1e-3) / 1e9,
+        "stage_gbs": {k_: sb[k_] / (stage_ms[k_] * 1e-3) / 1e9 for k_ in ("pool", "pack", "pack_pool", "merge")
+                      if k_ in stage_ms},
         "path": path,
         "roofline": {"kernel": ("bsa_block_sparse_attn_fused" if path == "fused" else "bsa_block_sparse_attn")
                                + " (tcgen05 attention)", "bound": "tensor",

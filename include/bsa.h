@@ -130,6 +130,19 @@ BSA_API bsa_status bsa_pack_qkv(const bsa_layout* layout, const void* q, const v
                         bsa_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
+ * Packing and step 1 in one pass: the packed workspace of bsa_pack_qkv and the pooled
+ * pq, pk of bsa_pool_qk (same layouts and values up to fp32 summation order), reading
+ * Q and K from HBM once for both. For f32 layouts only the pooling runs (workspace
+ * ignored, may be NULL).
+ *   q, k, v          : device, [N, H, d] of layout->dtype
+ *   workspace        : bf16: device, at least bsa_workspace_size() bytes, 1024-byte aligned
+ *   pq, pk           : device, float32 [H, B, d] and [H, d, B]
+ */
+BSA_API bsa_status bsa_pack_pool_qkv(const bsa_layout* layout, const void* q, const void* k,
+                             const void* v, void* workspace, size_t workspace_bytes,
+                             float* pq, float* pk, int32_t* status_dev, bsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
  * Step 4 -- block-sparse attention over the selected blocks (关键设计 1, Eq. (2)).
  * For every head h and patch token p of query block i:
  *   o_pp[p, h, :] = softmax over the patch keys of the blocks kv_idx[h, i, :kv_cnt[h,i]]

@@ -55,7 +55,17 @@ def run_gpu(w: configs.Workload, x: synth.LayerInputs, density=None, tamper=None
         kv_idx=L.buf.kv_idx.cpu().numpy().view(np.uint16), kv_cnt=L.buf.kv_cnt.cpu().numpy(),
         pq=L.buf.pq.cpu().numpy(), pk=L.buf.pk.cpu().numpy(),
         o_pp=L.buf.o_pp.cpu().numpy(), lse_pp=L.buf.lse_pp.cpu().numpy(),
-        o_ps=L.buf.o_ps.cpu().numpy(), lse_ps=L.buf.lse_ps.cpu().numpy())
+        o_ps=L.buf.o_ps.cpu().numpy(), lse_ps=L.buf.lse_ps.cpu().numpy(), forward=None)
+    if w.dtype == "bf16":
+        # the whole layer through forward(): one-pass packing + pooling, mask, fused attention
+        L.buf.pq.zero_()
+        L.buf.pk.zero_()
+        L.buf.out.zero_()
+        L.forward(q, k, v)
+        torch.cuda.synchronize()
+        res["status"] = res["status"] or L.check_status()
+        res["forward"] = dict(pq=L.buf.pq.cpu().numpy(), pk=L.buf.pk.cpu().numpy(), selected=L.selected(),
+                              out=L.buf.out.float().cpu().numpy())
     return res
 
 

@@ -73,7 +73,9 @@ def test_perhead_budgets(lib):
 def test_workspace_size(lib):
     w = configs.PERHEAD100
     n = _lib.bsa_workspace_size(_lib.layout_of(w))
-    np_pad, ns_pad, nsplit = 77824, 512, 10        # key-range splits: ceil((4 + 608) / 64)
+    # key-range splits of the 512 special queries (4 tiles x 16 heads = 64 CTAs per split)
+    # over 4 + 608 key tiles: 9 splits fill 576 of the 592 slots of two waves (97%)
+    np_pad, ns_pad, nsplit = 77824, 512, 9
     assert n == 3 * 16 * (np_pad + ns_pad) * 128 + nsplit * 16 * ns_pad * (64 + 1) * 4
     assert _lib.bsa_workspace_size(_lib.layout_of(configs.TINY)) == 0
 
@@ -121,6 +123,16 @@ def test_step_argument_validation(lib):
     assert lib.bsa_block_sparse_attn(lay, A, A, A, None, 0, A, A, A, None, None, None) == E.BSA_ERR_INVALID_ARG
     assert lib.bsa_special_dense(lay, A, A, A, None, 0, None, None, None, None, None) == E.BSA_ERR_INVALID_ARG
     assert lib.bsa_merge(lay, A, A, A, A, None, None, None) == E.BSA_ERR_INVALID_ARG
+    # one-pass packing + pooling: pooled outputs required; bf16 also needs V and the workspace
+    assert lib.bsa_pack_pool_qkv(lay, A, A, A, None, 0, None, A, None, None) == E.BSA_ERR_INVALID_ARG
+    assert lib.bsa_pack_pool_qkv(lay, A, A + 8, A, None, 0, A, A, None, None) == E.BSA_ERR_INVALID_ARG
+    bf = _lay(dtype="bf16", block=64)
+    ws = ctypes.c_size_t()
+    assert lib.bsa_workspace_size(ctypes.byref(bf), ctypes.byref(ws)) == E.BSA_OK and ws.value > 0
+    bfr = ctypes.byref(bf)
+    assert lib.bsa_pack_pool_qkv(bfr, A, A, None, A, ws.value, A, A, None, None) == E.BSA_ERR_INVALID_ARG
+    assert lib.bsa_pack_pool_qkv(bfr, A, A, A, None, ws.value, A, A, None, None) == E.BSA_ERR_INVALID_ARG
+    assert lib.bsa_pack_pool_qkv(bfr, A, A, A, A, ws.value - 1, A, A, None, None) == E.BSA_ERR_INVALID_ARG
     bf = _lay(dtype="bf16", block=64, tokens_per_frame=782, frames=4)
     ws = ctypes.c_size_t()
     assert lib.bsa_workspace_size(ctypes.byref(bf), ctypes.byref(ws)) == E.BSA_OK

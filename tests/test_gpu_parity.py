@@ -68,21 +68,36 @@ def test_mask_and_layer(w):
     # output, against the oracle fed the device mask
     Q, K, V = (exact(a, w.dtype) for a in (x.q, x.k, x.v))
     tol = F32_TOL if w.dtype == "f32" else BF16_TOL
-    if lay.N * lay.heads <= 4096:
-        ref = oracle.layer_forward(Q.astype(np.float64), K.astype(np.float64), V.astype(np.float64),
-                                   lay, res["selected"])
-        pick = lambda a: a
+    small = lay.N * lay.heads <= 4096
+    rows, heads = (None, None) if small else sample_pairs(w, 2048)
+
+    def reference(selected):
+        if small:
+            return oracle.layer_forward(Q.astype(np.float64), K.astype(np.float64), V.astype(np.float64),
+                                        lay, selected)
+        return oracle.layer_rows(Q, K, V, lay, selected, rows, heads)
+
+    pick = (lambda a: a) if small else (lambda a: a[rows, heads])
+    ref = reference(res["selected"])
+    if small:
         print(f"{w.name}: nmse/head {nmse_per_head(res['out'], ref)}")
-    else:
-        rows, heads = sample_pairs(w, 2048)
-        ref = oracle.layer_rows(Q, K, V, lay, res["selected"], rows, heads)
-        pick = lambda a: a[rows, heads]
     for key in ("out", "out_fused"):
         if res[key] is None:
             continue
         got = pick(res[key])
         e2, ea = rel_l2(got, ref), max_abs(got, ref)
         print(f"{w.name} {key}: rel_l2 {e2:.3e} max_abs {ea:.3e}")
+        assert e2 <= tol[0] and ea <= tol[1]
+    # forward(): pooling folded into the packing pass, then mask and fused attention
+    fwd = res["forward"]
+    if fwd is not None:
+        assert max_abs(fwd["pq"], PQ) < 1e-5 and max_abs(fwd["pk"], PK.transpose(0, 2, 1)) < 1e-5
+        rep = compare_mask(om, fwd["selected"], w.tau)
+        assert rep.ok, rep.failures
+        ref_f = ref if np.array_equal(fwd["selected"], res["selected"]) else reference(fwd["selected"])
+        got = pick(fwd["out"])
+        e2, ea = rel_l2(got, ref_f), max_abs(got, ref_f)
+        print(f"{w.name} forward: rel_l2 {e2:.3e} max_abs {ea:.3e}")
         assert e2 <= tol[0] and ea <= tol[1]
 
 

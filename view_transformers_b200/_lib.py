@@ -37,6 +37,7 @@ _SIGS = {
     "bsa_pool_qk": [_LP, _vp, _vp, _vp, _vp, _i32p, _st],
     "bsa_predict_mask": [_LP, _vp, _vp, ctypes.c_double, ctypes.c_double, ctypes.c_void_p, _vp, _vp, _vp, _i32p, _st],
     "bsa_pack_qkv": [_LP, _vp, _vp, _vp, _vp, _sz, _i32p, _st],
+    "bsa_pack_pool_qkv": [_LP, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _i32p, _st],
     "bsa_block_sparse_attn": [_LP, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp, _vp, _i32p, _st],
     "bsa_special_dense": [_LP, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp, _i32p, _st],
     "bsa_merge": [_LP, _vp, _vp, _vp, _vp, _vp, _i32p, _st],
@@ -153,6 +154,11 @@ def bsa_predict_mask(layout, pq, pk, rho, tau, head_density, mask_bits, kv_idx, 
 def bsa_pack_qkv(layout, q, k, v, workspace, workspace_bytes, status=0, stream=0) -> None:
     _check("bsa_pack_qkv", load().bsa_pack_qkv(ctypes.byref(layout), q, k, v, workspace, workspace_bytes,
                                                status, stream))
+
+
+def bsa_pack_pool_qkv(layout, q, k, v, workspace, workspace_bytes, pq, pk, status=0, stream=0) -> None:
+    _check("bsa_pack_pool_qkv", load().bsa_pack_pool_qkv(ctypes.byref(layout), q, k, v, workspace,
+                                                         workspace_bytes, pq, pk, status, stream))
 
 
 def bsa_block_sparse_attn(layout, q, k, v, workspace, workspace_bytes, kv_idx, kv_cnt, o_pp, lse_pp,

@@ -26,6 +26,8 @@ int num_sms() {
 cudaError_t launch_attn_tc(const Geo& g, int mode, const void* ws, const uint16_t* kv_idx,
                            const int32_t* kv_cnt, float* o_part, float* lse_part, void* out,
                            int32_t* status, cudaStream_t st);
+cudaError_t launch_pack_pool(const Geo& g, const void* q, const void* k, const void* v, void* ws,
+                             float* pq, float* pk, cudaStream_t st);
 cudaError_t launch_pack(const Geo& g, const void* q, const void* k, const void* v, void* ws,
                         cudaStream_t st);
 
@@ -134,6 +136,28 @@ bsa_status bsa_pack_qkv(const bsa_layout* layout, const void* q, const void* k, 
     s = check_ws(g, workspace, workspace_bytes);
     if (s != BSA_OK) return s;
     return from_cuda(launch_pack(g, q, k, v, workspace, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+bsa_status bsa_pack_pool_qkv(const bsa_layout* layout, const void* q, const void* k, const void* v,
+                             void* workspace, size_t workspace_bytes, float* pq, float* pk,
+                             int32_t* status_dev, bsa_stream_t stream) {
+    (void)status_dev;
+    Geo g;
+    bsa_status s = make_geo(layout, &g);
+    if (s != BSA_OK) return s;
+    if (!q || !k || !pq || !pk) return BSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(pq) || !aligned16(pk)) return BSA_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (layout->dtype != BSA_BF16) return from_cuda(launch_pool(g, layout->dtype, q, k, pq, pk, st));
+    if (!v || !aligned16(v)) return BSA_ERR_INVALID_ARG;
+    s = check_ws(g, workspace, workspace_bytes);
+    if (s != BSA_OK) return s;
+    if (!tc_supported(g)) {   // the one-pass kernel needs whole blocks per 128-row tile
+        cudaError_t e = launch_pack(g, q, k, v, workspace, st);
+        if (e == cudaSuccess) e = launch_pool(g, layout->dtype, q, k, pq, pk, st);
+        return from_cuda(e);
+    }
+    return from_cuda(launch_pack_pool(g, q, k, v, workspace, pq, pk, st));
 }
 
 bsa_status bsa_k_from_rho(int32_t num_blocks, double rho, int32_t* k) {

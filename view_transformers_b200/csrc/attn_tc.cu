@@ -166,10 +166,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int sp_tiles = (g.Ns + BKV - 1) / BKV;   // special key tiles (BKV rows)
     int t_begin = 0, t_end = 0;                    // MODE_SPECIAL_ALL key-tile range
     if (MODE == MODE_SPECIAL_ALL) {
-        const int n_all = sp_tiles + pl.np_pad / 128;
-        const int chunk = (n_all + pl.nsplit - 1) / pl.nsplit;
-        t_begin = min(n_all, split * chunk);
-        t_end = min(n_all, t_begin + chunk);
+        const int n_all = sp_tiles + pl.np_pad / 128;   // even split: sizes differ by at most one
+        t_begin = (int)((long long)split * n_all / pl.nsplit);
+        t_end = (int)((long long)(split + 1) * n_all / pl.nsplit);
     }
 
     // ------------------------------------------------------------------ setup

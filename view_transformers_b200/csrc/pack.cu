@@ -66,6 +66,116 @@ pack_kernel(Geo g, PackedLayout pl, const __nv_bfloat16* __restrict__ q,
     }
 }
 
+// Packing with block pooling folded in: the same copies as pack_kernel, plus the block
+// means P_b(Q), P_b(K) of 关键设计 1 taken from the patch rows while they pass through
+// registers, so Q and K are read from HBM once for both steps. Written for b dividing 128
+// (64 or 128): a 128-row tile then holds 128 / b whole blocks.
+//
+// Work unit: one 128-row tile (patch tiles first, then special tiles) x one group of 4
+// heads. 256 threads = 32 chunks of 16 bytes (4 heads x 8) x 8 row phases of 16
+// consecutive rows; a row phase therefore never straddles a block. Each thread sums its 16
+// rows in fp32 in row order, then the phases of a block are added in phase order, so the
+// pooled values do not depend on scheduling.
+constexpr int kPoolHeads = 4;                 // heads per work unit
+constexpr int kPhaseRows = 16;                // consecutive rows per thread
+constexpr int kPhases = 128 / kPhaseRows;     // row phases per tile
+
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 w) {
+    const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __half2 hv = __floats2half2_rn(__uint_as_float(in[i] << 16), __uint_as_float(in[i] & 0xffff0000u));
+        o[i] = *reinterpret_cast<const uint32_t*>(&hv);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__device__ __forceinline__ void add_bf16x8(float* acc, uint4 w) {
+    const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        acc[2 * i] += __uint_as_float(in[i] << 16);
+        acc[2 * i + 1] += __uint_as_float(in[i] & 0xffff0000u);
+    }
+}
+
+__global__ void __launch_bounds__(256)
+pack_pool_kernel(Geo g, PackedLayout pl, const __nv_bfloat16* __restrict__ q,
+                 const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+                 unsigned char* __restrict__ ws, float* __restrict__ pq, float* __restrict__ pk) {
+    __shared__ float red[2][kPhases][kPoolHeads * 64];   // per-phase sums of Q and K
+    const int groups = (g.H + kPoolHeads - 1) / kPoolHeads;
+    const int p_tiles = pl.np_pad / 128;
+    const int units = (p_tiles + pl.ns_pad / 128) * groups;
+    const int c = threadIdx.x % (kPoolHeads * 8);       // chunk within the head group
+    const int ph = threadIdx.x / (kPoolHeads * 8);      // row phase
+    const int c8 = c & 7;
+    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+        const int tile = u / groups;
+        const int h = (u - tile * groups) * kPoolHeads + (c >> 3);
+        const bool patch = tile < p_tiles;
+        const bool active = h < g.H;
+        const int r0 = (patch ? tile : tile - p_tiles) * 128 + ph * kPhaseRows;
+        float sq[8], sk[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) { sq[e] = 0.f; sk[e] = 0.f; }
+        if (active) {
+            const int limit = patch ? g.Np : g.Ns;
+            const size_t dst_base = (size_t)h * (patch ? pl.np_pad : pl.ns_pad);
+            unsigned char* oq = ws + (patch ? pl.qp : pl.qs);
+            unsigned char* ok = ws + (patch ? pl.kp : pl.ks);
+            unsigned char* ov = ws + (patch ? pl.vp : pl.vs);
+#pragma unroll 4
+            for (int i = 0; i < kPhaseRows; ++i) {
+                const int r = r0 + i;
+                uint4 vq = make_uint4(0, 0, 0, 0), vk = vq, vv = vq;
+                if (r < limit) {
+                    const int src_row = patch ? patch_row(g, r) : special_row(g, r);
+                    const size_t off = (size_t)src_row * g.H * 64 + (size_t)h * 64 + c8 * 8;
+                    vq = __ldg(reinterpret_cast<const uint4*>(q + off));
+                    vk = __ldg(reinterpret_cast<const uint4*>(k + off));
+                    vv = bf16x8_to_f16x8(__ldg(reinterpret_cast<const uint4*>(v + off)));
+                    if (patch) { add_bf16x8(sq, vq); add_bf16x8(sk, vk); }
+                }
+                const size_t dst = (dst_base + r) * 128 + c8 * 16;
+                *reinterpret_cast<uint4*>(oq + dst) = vq;
+                *reinterpret_cast<uint4*>(ok + dst) = vk;
+                *reinterpret_cast<uint4*>(ov + dst) = vv;
+            }
+        }
+        if (patch) {   // the same for the whole CTA
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                red[0][ph][c * 8 + e] = sq[e];
+                red[1][ph][c * 8 + e] = sk[e];
+            }
+            __syncthreads();
+            const int per_tile = 128 / g.b;            // whole blocks in the tile
+            const int pb = kPhases / per_tile;         // row phases per block
+            const int h0 = (u - tile * groups) * kPoolHeads;
+            constexpr int kOut = 2 * kPoolHeads * 64;  // (Q|K) x head x dimension
+            for (int x = threadIdx.x; x < per_tile * kOut; x += blockDim.x) {
+                const int blk = x / kOut;
+                const int t = (x - blk * kOut) / (kPoolHeads * 64);   // 0: Q, 1: K
+                const int e = x - blk * kOut - t * kPoolHeads * 64;  // head in group x 64 + dim
+                const int j = tile * per_tile + blk;
+                const int hh = h0 + e / 64;
+                if (j < g.B && hh < g.H) {
+                    float sum = 0.f;
+                    for (int p2 = blk * pb; p2 < (blk + 1) * pb; ++p2) sum += red[t][p2][e];
+                    const int lo = j * g.b;
+                    const int hi = min(lo + g.b, g.Np);
+                    const float mean = sum / (float)(hi - lo);
+                    const int dd = e & 63;
+                    if (t == 0) pq[((size_t)hh * g.B + j) * 64 + dd] = mean;   // [H][B][d]
+                    else pk[((size_t)hh * 64 + dd) * g.B + j] = mean;          // [H][d][B]
+                }
+            }
+            __syncthreads();
+        }
+    }
+}
 }  // namespace
 
 cudaError_t launch_pack(const Geo& g, const void* q, const void* k, const void* v, void* ws,
@@ -75,6 +185,21 @@ cudaError_t launch_pack(const Geo& g, const void* q, const void* k, const void* 
                                                static_cast<const __nv_bfloat16*>(k),
                                                static_cast<const __nv_bfloat16*>(v),
                                                static_cast<unsigned char*>(ws));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack_pool(const Geo& g, const void* q, const void* k, const void* v, void* ws,
+                             float* pq, float* pk, cudaStream_t st) {
+    const PackedLayout pl = packed_layout(g);
+    const int groups = (g.H + kPoolHeads - 1) / kPoolHeads;
+    const int units = (pl.np_pad / 128 + pl.ns_pad / 128) * groups;
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pack_pool_kernel, 256, 0);
+    if (e != cudaSuccess) return e;
+    const int slots = num_sms() * (per_sm > 0 ? per_sm : 1);
+    pack_pool_kernel<<<units < slots ? units : slots, 256, 0, st>>>(
+        g, pl, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+        static_cast<const __nv_bfloat16*>(v), static_cast<unsigned char*>(ws), pq, pk);
     return cudaGetLastError();
 }
 

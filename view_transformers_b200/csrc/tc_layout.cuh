@@ -20,13 +20,35 @@ struct PackedLayout {
     size_t bytes;        // total
 };
 
+// Key-range splits of the special-query attention (units = query tiles x heads CTAs per
+// split, n_all key tiles): the fewest splits, at most 128 key tiles each, whose CTAs fill
+// at least 95% of their last wave on a B200 (148 SMs, 2 attention CTAs resident per SM);
+// each split keeps at least 8 key tiles, and the best fill found is taken when none reaches
+// 95%.
+__host__ __device__ inline int special_splits(int units, int n_all) {
+    constexpr int kSlots = 148 * 2;
+    const int lo = (n_all + 127) / 128 > 1 ? (n_all + 127) / 128 : 1;
+    int hi = n_all / 8 < 64 ? n_all / 8 : 64;
+    hi = hi > lo ? hi : lo;
+    int best = lo;
+    double best_fill = 0.0;
+    for (int ns = lo; ns <= hi; ++ns) {
+        const long long ctas = (long long)units * ns;
+        const long long waves = (ctas + kSlots - 1) / kSlots;
+        const double fill = (double)ctas / (double)(waves * kSlots);
+        if (fill >= 0.95) return ns;
+        if (fill > best_fill) { best = ns; best_fill = fill; }
+    }
+    return best;
+}
+
 __host__ __device__ inline PackedLayout packed_layout(const Geo& g) {
     PackedLayout pl;
     pl.np_pad = (g.Np + 127) / 128 * 128;
     pl.ns_pad = (g.Ns + 127) / 128 * 128;
-    // special queries see every key: split the key range into chunks of about 64 tiles
+    // special queries see every key: the key range is split across CTAs
     const int n_all = pl.ns_pad / 128 + pl.np_pad / 128;
-    pl.nsplit = g.Ns == 0 ? 0 : (n_all + 63) / 64 > 16 ? 16 : (n_all + 63) / 64;
+    pl.nsplit = g.Ns == 0 ? 0 : special_splits(pl.ns_pad / 128 * g.H, n_all);
     const size_t patch = (size_t)g.H * pl.np_pad * 128;
     const size_t spec = (size_t)g.H * pl.ns_pad * 128;
     pl.qp = 0;

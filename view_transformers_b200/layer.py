@@ -112,10 +112,26 @@ class BlockSparseLayer:
                 fused: bool | None = None) -> torch.Tensor:
         """The whole layer: [N, H, d] tensors in the layer dtype, on this device. bf16 layers
         use the fused patch-row pass unless fused=False."""
-        self.predict(q, k, stream)
         if fused is None:
             fused = self.dtype == "bf16"
-        return self.attend_fused(q, k, v, stream) if fused else self.attend(q, k, v, stream)
+        if not fused:
+            self.predict(q, k, stream)
+            return self.attend(q, k, v, stream)
+        st = self._stream(stream)
+        b = self.buf
+        qp, kp, vp = q.data_ptr(), k.data_ptr(), v.data_ptr()
+        # packing and pooling in one pass over Q, K, V; then mask, special rows, patch rows
+        _lib.bsa_pack_pool_qkv(self.layout, qp, kp, vp, self.ws_ptr, self.ws_bytes, b.pq.data_ptr(),
+                               b.pk.data_ptr(), b.status.data_ptr(), st)
+        _lib.bsa_predict_mask(self.layout, b.pq.data_ptr(), b.pk.data_ptr(), self.rho, self.tau,
+                              self.head_density, b.mask_bits.data_ptr(), b.kv_idx.data_ptr(),
+                              b.kv_cnt.data_ptr(), b.status.data_ptr(), st)
+        _lib.bsa_special_dense(self.layout, qp, kp, vp, self.ws_ptr, self.ws_bytes, b.out.data_ptr(),
+                               None, None, b.status.data_ptr(), st)
+        _lib.bsa_block_sparse_attn_fused(self.layout, qp, kp, vp, self.ws_ptr, self.ws_bytes,
+                                         b.kv_idx.data_ptr(), b.kv_cnt.data_ptr(), b.out.data_ptr(),
+                                         b.status.data_ptr(), st)
+        return b.out
 
     def check_status(self, stream: int | None = None) -> int:
         return _lib.bsa_check_status(self.buf.status.data_ptr(), self._stream(stream))
