@@ -373,17 +373,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             // s[2i+1] were read
             float rs = 0.f;
             if (full) {
-                float r[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // independent partial sums
+                // packed fp32 pair arithmetic: half the issue slots of scalar FMA / add
+                float2 r2[4];   // independent partial sums
+#pragma unroll
+                for (int i = 0; i < 4; ++i) r2[i] = make_float2(0.f, 0.f);
+                const float2 scale2 = make_float2(kScaleLog2, kScaleLog2);
+                const float2 shift2 = make_float2(-m_ref, -m_ref);
 #pragma unroll
                 for (int c = 0; c < BKV; c += 2) {
-                    const float p0 = ex2_approx(fmaf(__uint_as_float(s[c]), kScaleLog2, -m_ref));
-                    const float p1 = ex2_approx(fmaf(__uint_as_float(s[c + 1]), kScaleLog2, -m_ref));
-                    r[(c / 2) & 3] += p0;
-                    r[((c / 2) & 3) + 4] += p1;
-                    const __half2 hp = __floats2half2_rn(p0, p1);
-                    s[c / 2] = *reinterpret_cast<const uint32_t*>(&hp);
+                    const int i = c / 2;
+                    const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
+                                                scale2, shift2);
+                    const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                    r2[i & 3] = __fadd2_rn(r2[i & 3], pr);
+                    s[i] = pack_half2(pr.x, pr.y);   // pair i lands in s[i] after s[2i], s[2i+1] were read
                 }
-                rs = ((r[0] + r[1]) + (r[2] + r[3])) + ((r[4] + r[5]) + (r[6] + r[7]));
+                rs = ((r2[0].x + r2[0].y) + (r2[1].x + r2[1].y)) + ((r2[2].x + r2[2].y) + (r2[3].x + r2[3].y));
             } else {
 #pragma unroll
                 for (int c = 0; c < BKV; c += 2) {
