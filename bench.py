@@ -1,7 +1,9 @@
 """Benchmark of the block-sparse global-attention layer on B200.
 
-One step = one whole layer on one GPU: pool -> mask -> pack -> special dense ->
-block-sparse attention -> merge, on seeded synthetic inputs already resident in HBM.
+One step = one whole layer on one GPU, on seeded synthetic inputs already resident in HBM.
+bf16 layers (default): packing + pooling -> mask -> special queries -> fused patch rows
+(block-sparse attention, special keys and the merge in one pass). `--path five`: pool ->
+mask -> pack -> special dense -> block-sparse attention -> merge.
 Default workload: 100 frames x (777 patch + 5 special) tokens, 16 heads, d = 64, b = 128,
 layer budget rho = 0.75 split across heads by capped water-filling of LogNormal(0, 1)
 scores, tau = 0.
@@ -280,6 +282,22 @@ def workload_config(w):
             "l2": "inputs larger than L2 (Q, K, V and the packed workspace: about 1 GB touched per step)"}
 
 
+# ---------------------------------------------------------------------------- ranks
+def max_over_ranks(value: float, dist, device) -> float:
+    """The job's time is its slowest rank's: max of a per-rank value over all ranks."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_ms_per_layer(total_ms_max: float, steps: int, world: int) -> float:
+    """Whole-job ms per layer: every rank runs `steps` layers (replicas, weak scaling)."""
+    return total_ms_max / (steps * world)
+
+
 # ---------------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -341,12 +359,9 @@ def main():
     torch.cuda.synchronize()
     status = L.check_status()
     clocks = clk.summary()
-    t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
-    if dist:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dist, "cuda")
     ms_per_step = total_ms / args.steps
-    value = total_ms / (args.steps * world)          # whole job: layers processed by all ranks
+    value = job_ms_per_layer(total_ms, args.steps, world)   # whole job: layers of all ranks
 
     kv_cnt = L.buf.kv_cnt.cpu().numpy()
     kv_idx = L.buf.kv_idx.cpu().numpy().view(np.uint16)
@@ -390,10 +405,7 @@ def main():
         s1.record()
         s1.synchronize()
         e2e_ms = s0.elapsed_time(s1) / args.e2e_steps
-    t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-    if dist:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_value = float(t.item()) / world
+    e2e_value = max_over_ranks(e2e_ms, dist, "cuda") / world
 
     hbm, tf_burst, tf_sus, peak_src = peaks()
     sparse_ms = stage_ms["sparse"]

@@ -238,6 +238,17 @@ BSA_API bsa_status bsa_attention_noalloc(const bsa_layout* layout, const void* q
                                          void* out, int32_t* status_dev, bsa_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
+ * Self-check of the bounded device waits (no counterpart on the pages). Launches one
+ * thread that waits, with the same bounded wait as the attention kernels, on an
+ * mbarrier that nothing arrives on. After limit_us microseconds the wait gives up and
+ * writes BSA_ERR_TIMEOUT to *status_dev; the kernel then returns normally and the
+ * context stays usable. Read the result with bsa_check_status.
+ *   status_dev : device int32, required
+ *   limit_us   : 1 .. 10,000,000
+ */
+BSA_API bsa_status bsa_selftest_wait_timeout(int32_t* status_dev, uint32_t limit_us, bsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
  * Host helpers (no device work).
  */
 /* B = ceil(F P / b). */

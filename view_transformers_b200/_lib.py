@@ -50,6 +50,7 @@ _SIGS = {
     "bsa_head_budgets": [ctypes.POINTER(ctypes.c_double), ctypes.c_int32, ctypes.c_double, ctypes.c_double,
                          ctypes.POINTER(ctypes.c_double)],
     "bsa_check_status": [_i32p, _st],
+    "bsa_selftest_wait_timeout": [_i32p, ctypes.c_uint32, _st],
     "bsa_status_string": [ctypes.c_int],
 }
 
@@ -128,6 +129,10 @@ def bsa_head_budgets(scores, rho: float, cap: float = 1.0) -> list[float]:
     d = (ctypes.c_double * n)()
     _check("bsa_head_budgets", load().bsa_head_budgets(s, n, rho, cap, d))
     return list(d)
+
+
+def bsa_selftest_wait_timeout(status_ptr: int, limit_us: int, stream: int = 0) -> None:
+    _check("bsa_selftest_wait_timeout", load().bsa_selftest_wait_timeout(status_ptr, limit_us, stream))
 
 
 def bsa_check_status(status_ptr: int, stream: int = 0) -> int:

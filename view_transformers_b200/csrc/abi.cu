@@ -206,6 +206,14 @@ bsa_status bsa_head_budgets(const double* scores, int32_t heads, double rho, dou
     return BSA_OK;
 }
 
+bsa_status bsa_selftest_wait_timeout(int32_t* status_dev, uint32_t limit_us, bsa_stream_t stream) {
+    if (status_dev == nullptr || (reinterpret_cast<uintptr_t>(status_dev) & 3u) != 0u || limit_us < 1u ||
+        limit_us > 10000000u)
+        return BSA_ERR_INVALID_ARG;
+    return from_cuda(launch_wait_timeout(status_dev, (uint64_t)limit_us * 1000ull,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
 bsa_status bsa_check_status(int32_t* status_dev, bsa_stream_t stream) {
     if (status_dev == nullptr) return BSA_ERR_INVALID_ARG;
     int32_t v = 0;

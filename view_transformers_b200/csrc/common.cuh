@@ -100,5 +100,6 @@ cudaError_t launch_attn_simt(const Geo& g, bsa_dtype dt, int mode, const void* q
 cudaError_t launch_merge(const Geo& g, bsa_dtype dt, const float* o_pp, const float* lse_pp,
                          const float* o_ps, const float* lse_ps, void* out, cudaStream_t st);
 cudaError_t launch_fill(float* p, size_t n, float value, cudaStream_t st);
+cudaError_t launch_wait_timeout(int32_t* status, uint64_t limit_ns, cudaStream_t st);
 int num_sms();
 }  // namespace bsa
