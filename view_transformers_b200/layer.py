@@ -80,19 +80,21 @@ class BlockSparseLayer:
                               self.head_density, b.mask_bits.data_ptr(), b.kv_idx.data_ptr(),
                               b.kv_cnt.data_ptr(), b.status.data_ptr(), st)
 
-    def attend(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream: int | None = None) -> torch.Tensor:
+    def attend(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream: int | None = None,
+               out: torch.Tensor | None = None) -> torch.Tensor:
         st = self._stream(stream)
         b = self.buf
+        o = self._out(out)
         qp, kp, vp = q.data_ptr(), k.data_ptr(), v.data_ptr()
         _lib.bsa_pack_qkv(self.layout, qp, kp, vp, self.ws_ptr, self.ws_bytes, b.status.data_ptr(), st)
-        _lib.bsa_special_dense(self.layout, qp, kp, vp, self.ws_ptr, self.ws_bytes, b.out.data_ptr(),
+        _lib.bsa_special_dense(self.layout, qp, kp, vp, self.ws_ptr, self.ws_bytes, o.data_ptr(),
                                b.o_ps.data_ptr(), b.lse_ps.data_ptr(), b.status.data_ptr(), st)
         _lib.bsa_block_sparse_attn(self.layout, qp, kp, vp, self.ws_ptr, self.ws_bytes, b.kv_idx.data_ptr(),
                                    b.kv_cnt.data_ptr(), b.o_pp.data_ptr(), b.lse_pp.data_ptr(),
                                    b.status.data_ptr(), st)
         _lib.bsa_merge(self.layout, b.o_pp.data_ptr(), b.lse_pp.data_ptr(), b.o_ps.data_ptr(),
-                       b.lse_ps.data_ptr(), b.out.data_ptr(), b.status.data_ptr(), st)
-        return b.out
+                       b.lse_ps.data_ptr(), o.data_ptr(), b.status.data_ptr(), st)
+        return o
 
     def attend_fused(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                      stream: int | None = None) -> torch.Tensor:
@@ -109,16 +111,18 @@ class BlockSparseLayer:
         return b.out
 
     def forward(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream: int | None = None,
-                fused: bool | None = None) -> torch.Tensor:
+                fused: bool | None = None, out: torch.Tensor | None = None) -> torch.Tensor:
         """The whole layer: [N, H, d] tensors in the layer dtype, on this device. bf16 layers
-        use the fused patch-row pass unless fused=False."""
+        use the fused patch-row pass unless fused=False. The result goes to `out` when given
+        (an [N, H, d] contiguous tensor of the layer dtype), else to the layer's own buffer."""
         if fused is None:
             fused = self.dtype == "bf16"
         if not fused:
             self.predict(q, k, stream)
-            return self.attend(q, k, v, stream)
+            return self.attend(q, k, v, stream, out)
         st = self._stream(stream)
         b = self.buf
+        o = self._out(out)
         qp, kp, vp = q.data_ptr(), k.data_ptr(), v.data_ptr()
         # packing and pooling in one pass over Q, K, V; then mask, special rows, patch rows
         _lib.bsa_pack_pool_qkv(self.layout, qp, kp, vp, self.ws_ptr, self.ws_bytes, b.pq.data_ptr(),
@@ -126,17 +130,26 @@ class BlockSparseLayer:
         _lib.bsa_predict_mask(self.layout, b.pq.data_ptr(), b.pk.data_ptr(), self.rho, self.tau,
                               self.head_density, b.mask_bits.data_ptr(), b.kv_idx.data_ptr(),
                               b.kv_cnt.data_ptr(), b.status.data_ptr(), st)
-        _lib.bsa_special_dense(self.layout, qp, kp, vp, self.ws_ptr, self.ws_bytes, b.out.data_ptr(),
+        _lib.bsa_special_dense(self.layout, qp, kp, vp, self.ws_ptr, self.ws_bytes, o.data_ptr(),
                                None, None, b.status.data_ptr(), st)
         _lib.bsa_block_sparse_attn_fused(self.layout, qp, kp, vp, self.ws_ptr, self.ws_bytes,
-                                         b.kv_idx.data_ptr(), b.kv_cnt.data_ptr(), b.out.data_ptr(),
+                                         b.kv_idx.data_ptr(), b.kv_cnt.data_ptr(), o.data_ptr(),
                                          b.status.data_ptr(), st)
-        return b.out
+        return o
 
     def check_status(self, stream: int | None = None) -> int:
         return _lib.bsa_check_status(self.buf.status.data_ptr(), self._stream(stream))
 
     # helpers ----------------------------------------------------------------------
+    def _out(self, out):
+        b = self.buf
+        if out is None:
+            return b.out
+        if (out.shape != b.out.shape or out.dtype != b.out.dtype or out.device != b.out.device
+                or not out.is_contiguous()):
+            raise ValueError(f"out must be a contiguous {tuple(b.out.shape)} {b.out.dtype} tensor on {b.out.device}")
+        return out
+
     def _stream(self, stream):
         return torch.cuda.current_stream(self.device).cuda_stream if stream is None else stream
 
