@@ -71,13 +71,14 @@ pack_kernel(Geo g, PackedLayout pl, const __nv_bfloat16* __restrict__ q,
 // registers, so Q and K are read from HBM once for both steps. Written for b dividing 128
 // (64 or 128): a 128-row tile then holds 128 / b whole blocks.
 //
-// Work unit: one 128-row tile (patch tiles first, then special tiles) x one group of 4
-// heads. 256 threads = 32 chunks of 16 bytes (4 heads x 8) x 8 row phases of 16
-// consecutive rows; a row phase therefore never straddles a block. Each thread sums its 16
+// Work unit (one CTA each): one 128-row tile (patch tiles first, then special tiles) x one
+// pair of heads. 256 threads = 16 chunks of 16 bytes (2 heads x 8) x 16 row phases of 8
+// consecutive rows; a row phase therefore never straddles a block. Each thread sums its 8
 // rows in fp32 in row order, then the phases of a block are added in phase order, so the
-// pooled values do not depend on scheduling.
-constexpr int kPoolHeads = 4;                 // heads per work unit
-constexpr int kPhaseRows = 16;                // consecutive rows per thread
+// pooled values do not depend on scheduling. Small units (thousands of CTAs) keep the HBM
+// queue full to the end of the pass.
+constexpr int kPoolHeads = 2;                 // heads per work unit
+constexpr int kPhaseRows = 8;                 // consecutive rows per thread
 constexpr int kPhases = 128 / kPhaseRows;     // row phases per tile
 
 __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 w) {
@@ -193,11 +194,7 @@ cudaError_t launch_pack_pool(const Geo& g, const void* q, const void* k, const v
     const PackedLayout pl = packed_layout(g);
     const int groups = (g.H + kPoolHeads - 1) / kPoolHeads;
     const int units = (pl.np_pad / 128 + pl.ns_pad / 128) * groups;
-    int per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pack_pool_kernel, 256, 0);
-    if (e != cudaSuccess) return e;
-    const int slots = num_sms() * (per_sm > 0 ? per_sm : 1);
-    pack_pool_kernel<<<units < slots ? units : slots, 256, 0, st>>>(
+    pack_pool_kernel<<<units, 256, 0, st>>>(
         g, pl, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
         static_cast<const __nv_bfloat16*>(v), static_cast<unsigned char*>(ws), pq, pk);
     return cudaGetLastError();

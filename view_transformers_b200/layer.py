@@ -111,10 +111,13 @@ class BlockSparseLayer:
         return b.out
 
     def forward(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream: int | None = None,
-                fused: bool | None = None, out: torch.Tensor | None = None) -> torch.Tensor:
+                fused: bool | None = None, out: torch.Tensor | None = None,
+                kernel_events=None) -> torch.Tensor:
         """The whole layer: [N, H, d] tensors in the layer dtype, on this device. bf16 layers
         use the fused patch-row pass unless fused=False. The result goes to `out` when given
-        (an [N, H, d] contiguous tensor of the layer dtype), else to the layer's own buffer."""
+        (an [N, H, d] contiguous tensor of the layer dtype), else to the layer's own buffer.
+        kernel_events: optional pair of CUDA events recorded on the calling stream right
+        before and after the patch-row attention launch (to time that kernel in place)."""
         if fused is None:
             fused = self.dtype == "bf16"
         if not fused:
@@ -124,7 +127,9 @@ class BlockSparseLayer:
         b = self.buf
         o = self._out(out)
         qp, kp, vp = q.data_ptr(), k.data_ptr(), v.data_ptr()
-        # packing and pooling in one pass over Q, K, V; then mask, special rows, patch rows
+        # packing and pooling in one pass over Q, K, V; then mask, special rows, patch rows.
+        # (Running the special rows on a second stream next to the mask and the patch rows
+        # was measured slower: both attention passes are compute-bound and share the SMs.)
         _lib.bsa_pack_pool_qkv(self.layout, qp, kp, vp, self.ws_ptr, self.ws_bytes, b.pq.data_ptr(),
                                b.pk.data_ptr(), b.status.data_ptr(), st)
         _lib.bsa_predict_mask(self.layout, b.pq.data_ptr(), b.pk.data_ptr(), self.rho, self.tau,
@@ -132,9 +137,15 @@ class BlockSparseLayer:
                               b.kv_cnt.data_ptr(), b.status.data_ptr(), st)
         _lib.bsa_special_dense(self.layout, qp, kp, vp, self.ws_ptr, self.ws_bytes, o.data_ptr(),
                                None, None, b.status.data_ptr(), st)
+        main = None
+        if kernel_events is not None:
+            main = torch.cuda.current_stream(self.device) if stream is None else torch.cuda.ExternalStream(stream)
+            kernel_events[0].record(main)
         _lib.bsa_block_sparse_attn_fused(self.layout, qp, kp, vp, self.ws_ptr, self.ws_bytes,
                                          b.kv_idx.data_ptr(), b.kv_cnt.data_ptr(), o.data_ptr(),
                                          b.status.data_ptr(), st)
+        if kernel_events is not None:
+            kernel_events[1].record(main)
         return o
 
     def check_status(self, stream: int | None = None) -> int:
