@@ -10,8 +10,10 @@
 //
 // Scores (FMA-bound): pooled K is stored dimension-major ([H][d][B]), so a warp reads 32
 // consecutive blocks of one dimension per load straight from L2; each lane accumulates
-// two blocks x R rows (2R independent FMA chains) with the R query values of a dimension
-// broadcast from shared memory, so one shared-memory wavefront feeds 8 FMAs per lane.
+// one block x 8 rows (8 independent FMA chains) with the query values of a dimension
+// broadcast from shared memory (one shared-memory wavefront feeds 4 FMAs per lane). The
+// small work items keep all 16 warps busy and the kernel within 64 registers, so two
+// CTAs share an SM.
 //
 // Selection: instead of sorting a row, a select over the fp32 scores in three steps:
 //   - one pass counts the row into 256 equal-width score buckets over [min, max] (with
@@ -382,7 +384,7 @@ __device__ void select_row(const float* s, int B, int h, int i, int k, double ta
 
 // R query-block rows i0 .. i0+R-1 of head h per CTA.
 template <int R>
-__global__ void __launch_bounds__(32 * kMaxWarps)
+__global__ void __launch_bounds__(32 * kMaxWarps, 2)
 mask_kernel(Geo g, MaskParams mp, const float* __restrict__ pq, const float* __restrict__ pk,
             uint32_t* __restrict__ mask_bits, uint16_t* __restrict__ kv_idx,
             int32_t* __restrict__ kv_cnt, int32_t* status) {
@@ -404,64 +406,57 @@ mask_kernel(Geo g, MaskParams mp, const float* __restrict__ pq, const float* __r
     }
     __syncthreads();
 
-    // ---- pooled scores: 64-block chunks round-robin over the warps
+    // ---- pooled scores: work items of 32 blocks (one per lane) x RG rows, round-robin over
+    // the warps (consecutive warps take consecutive block chunks)
+    constexpr int RG = R < 8 ? R : 8;
     const float* pk_h = pk + (size_t)h * kDim * B;
     const float scale = 0.125f;   // 1 / sqrt(64)
-    const int nchunk = (B + 63) / 64;
-    for (int c = warp; c < nchunk; c += W) {
-        const int j0 = c * 64 + lane;
-        const int j1 = j0 + 32;
-        const bool v0 = j0 < B, v1 = j1 < B;
-        const float* p0 = pk_h + (v0 ? j0 : 0);
-        const float* p1 = pk_h + (v1 ? j1 : 0);
-        float a0[R], a1[R];
+    const int nchunk = (B + 31) / 32;
+    const int items = nchunk * (R / RG);
+    for (int it = warp; it < items; it += W) {
+        const int c = it % nchunk;
+        const int rg = it / nchunk;
+        const int j = c * 32 + lane;
+        const bool valid = j < B;
+        const float* p = pk_h + (valid ? j : 0);
+        float a[RG];
 #pragma unroll
-        for (int r = 0; r < R; ++r) { a0[r] = 0.f; a1[r] = 0.f; }
-        float k0[8], k1[8];
+        for (int r = 0; r < RG; ++r) a[r] = 0.f;
+        float kc[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            k0[u] = __ldg(p0 + (size_t)u * B);
-            k1[u] = __ldg(p1 + (size_t)u * B);
-        }
+        for (int u = 0; u < 8; ++u) kc[u] = __ldg(p + (size_t)u * B);
 #pragma unroll 1
         for (int d0 = 0; d0 < kDim; d0 += 8) {
-            float n0[8], n1[8];
+            float kn[8];
             if (d0 + 8 < kDim) {   // next eight dimensions in flight during this group's FMAs
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    n0[u] = __ldg(p0 + (size_t)(d0 + 8 + u) * B);
-                    n1[u] = __ldg(p1 + (size_t)(d0 + 8 + u) * B);
-                }
+                for (int u = 0; u < 8; ++u) kn[u] = __ldg(p + (size_t)(d0 + 8 + u) * B);
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const float* qd = qT + (d0 + u) * R;
+                const float* qd = qT + (d0 + u) * R + rg * RG;
 #pragma unroll
-                for (int r4 = 0; r4 < R; r4 += (R >= 4 ? 4 : R)) {
+                for (int r4 = 0; r4 < RG; r4 += (RG >= 4 ? 4 : RG)) {
                     float qv[4];
-                    if constexpr (R >= 4) {
+                    if constexpr (RG >= 4) {
                         const float4 t = *reinterpret_cast<const float4*>(qd + r4);
                         qv[0] = t.x; qv[1] = t.y; qv[2] = t.z; qv[3] = t.w;
                     } else {
 #pragma unroll
-                        for (int e = 0; e < R; ++e) qv[e] = qd[e];
+                        for (int e = 0; e < RG; ++e) qv[e] = qd[e];
                     }
 #pragma unroll
-                    for (int e = 0; e < (R >= 4 ? 4 : R); ++e) {
-                        a0[r4 + e] = fmaf(qv[e], k0[u], a0[r4 + e]);
-                        a1[r4 + e] = fmaf(qv[e], k1[u], a1[r4 + e]);
-                    }
+                    for (int e = 0; e < (RG >= 4 ? 4 : RG); ++e) a[r4 + e] = fmaf(qv[e], kc[u], a[r4 + e]);
                 }
             }
             if (d0 + 8 < kDim) {
 #pragma unroll
-                for (int u = 0; u < 8; ++u) { k0[u] = n0[u]; k1[u] = n1[u]; }
+                for (int u = 0; u < 8; ++u) kc[u] = kn[u];
             }
         }
+        if (valid) {
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
-            if (v0) sc[(size_t)r * B + j0] = a0[r] * scale;
-            if (v1) sc[(size_t)r * B + j1] = a1[r] * scale;
+            for (int r = 0; r < RG; ++r) sc[(size_t)(rg * RG + r) * B + j] = a[r] * scale;
         }
     }
     __syncthreads();
