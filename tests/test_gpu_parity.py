@@ -145,6 +145,11 @@ EDGE = [
     configs.Workload("dense_rho0", 2, 300, 5, 2, 64, 64, 0.0, 0.0, "bf16", "five_percent"),
     configs.Workload("f32_ragged", 3, 37, 4, 2, 64, 10, 0.6, 0.3, "f32", "tiny"),
     configs.Workload("f32_no_special", 2, 40, 0, 2, 64, 16, 0.5, 0.5, "f32", "tiny"),
+    # a last block of one token, and a block count just above a multiple of 32
+    configs.Workload("tail1_b64", 3, 43, 5, 2, 64, 64, 0.5, 0.0, "bf16", "five_percent"),
+    configs.Workload("tail1_b128", 1, 129, 5, 2, 64, 128, 0.5, 0.0, "bf16", "five_percent"),
+    configs.Workload("b33_blocks", 3, 703, 5, 2, 64, 64, 0.6, 0.0, "bf16", "five_percent"),
+    configs.Workload("f32_tail1", 3, 11, 4, 2, 64, 16, 0.5, 0.3, "f32", "tiny"),
 ]
 
 
