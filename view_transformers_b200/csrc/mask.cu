@@ -48,8 +48,9 @@ struct WarpHist {
     unsigned long long mass[kRadix];
 };
 
+// Order-preserving 32-bit image of a score; -0 and +0 (equal scores) map to one key.
 __device__ __forceinline__ uint32_t order_key(float s) {
-    const uint32_t u = __float_as_uint(s);
+    const uint32_t u = __float_as_uint(s + 0.0f);
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
@@ -269,17 +270,18 @@ __device__ void select_row(const float* s, int B, int h, int i, int k, double ta
                            WarpHist* hist, uint32_t* __restrict__ mask_bits,
                            uint16_t* __restrict__ kv_idx, int32_t* __restrict__ kv_cnt,
                            int32_t* status, int lane) {
-    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    float fmin = FLT_MAX, fmax = -FLT_MAX;
     for (int j = lane; j < B; j += 32) {
-        const uint32_t u = order_key(s[j]);
-        kmin = min(kmin, u);
-        kmax = max(kmax, u);
+        const float sj = s[j];
+        fmin = fminf(fmin, sj);
+        fmax = fmaxf(fmax, sj);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-        kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
-        kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+        fmin = fminf(fmin, __shfl_xor_sync(0xffffffffu, fmin, o));
+        fmax = fmaxf(fmax, __shfl_xor_sync(0xffffffffu, fmax, o));
     }
+    const uint32_t kmin = order_key(fmin), kmax = order_key(fmax);
     const float mx = key_value(kmax);
     const float smin = key_value(kmin);
     const float scale = (float)kRadix / (mx - smin);
@@ -362,15 +364,16 @@ __device__ void select_row(const float* s, int B, int h, int i, int k, double ta
     const int words = (B + 31) / 32;
     uint16_t* out_idx = kv_idx + ((size_t)h * B + i) * B;
     int taken_ties = 0, written = 0;
+    const float tval = key_value(cut.t);   // score comparisons agree with key comparisons
     for (int j0 = 0; j0 < B; j0 += 32) {
         const int j = j0 + lane;
-        const bool valid = j < B;
-        const uint32_t u = valid ? order_key(s[j]) : 0u;
-        const bool tie = valid && !none && u == cut.t;
+        const bool valid = j < B && !none;
+        const float sj = valid ? s[j] : 0.f;
+        const bool tie = valid && sj == tval;
         const unsigned tb = __ballot_sync(0xffffffffu, tie);
         const int trank = taken_ties + __popc(tb & lanemask_lt());
         taken_ties += __popc(tb);
-        const bool sel = valid && !none && (u > cut.t || (tie && trank < cut.take));
+        const bool sel = valid && (sj > tval || (tie && trank < cut.take));
         const unsigned sb = __ballot_sync(0xffffffffu, sel);
         if (sel) out_idx[written + __popc(sb & lanemask_lt())] = (uint16_t)j;
         written += __popc(sb);

@@ -4,16 +4,18 @@
 //
 // HBM-bound: every patch row of Q and K is read once (Np * H * d elements each), the
 // pooled fp32 tensors are written once: pq as [H, B, d], pk dimension-major as [H, d, B]
-// (the layout the score pass of the mask kernel reads with coalesced loads). One CTA per (block, Q|K); each warp
-// reads whole 16-byte chunks of consecutive rows (a row holds all heads, 2 KB in bf16
-// at H = 16), so every load is a coalesced 512-byte warp transaction. Row groups inside
-// the CTA keep 8-16 independent 16-byte loads in flight per thread.
+// (the layout the score pass of the mask kernel reads with coalesced loads).
+// One CTA per (block, Q|K, 32 16-byte chunks of the row = 4 heads in bf16): thousands of
+// small CTAs keep the HBM queue full to the end. A warp reads 32 consecutive chunks of a
+// row (one coalesced 512-byte transaction); 8 row groups x 4 independent loads per thread
+// keep the loads in flight.
 #include "common.cuh"
 
 namespace bsa {
 namespace {
 
 constexpr int kPoolThreads = 256;
+constexpr int kChunksPerCta = 32;   // 16-byte chunks of a row per CTA (4 heads in bf16)
 
 template <typename T>
 __global__ void __launch_bounds__(kPoolThreads)
@@ -26,7 +28,9 @@ pool_kernel(Geo g, const T* __restrict__ q, const T* __restrict__ k, float* __re
     float* dst = blockIdx.y == 0 ? pq : pk;
     const int row_elems = g.H * g.d;
     const int chunks = row_elems / V;                     // 16-byte chunks per row
-    const int per_round = min(chunks, kPoolThreads);      // chunks covered per round
+    const int cbeg = blockIdx.z * kChunksPerCta;          // this CTA's chunks of every row
+    const int cend = min(chunks, cbeg + kChunksPerCta);
+    const int per_round = min(cend - cbeg, kPoolThreads); // chunks covered per round
     const int ngroups = kPoolThreads / per_round;         // row groups per round
     const int lo = j * g.b;
     const int hi = min(lo + g.b, g.Np);
@@ -34,9 +38,9 @@ pool_kernel(Geo g, const T* __restrict__ q, const T* __restrict__ k, float* __re
     const int gi = threadIdx.x / per_round;
     const int ci = threadIdx.x % per_round;
 
-    for (int c0 = 0; c0 < chunks; c0 += per_round) {
+    for (int c0 = cbeg; c0 < cend; c0 += per_round) {
         const int c = c0 + ci;
-        if (gi < ngroups && c < chunks) {
+        if (gi < ngroups && c < cend) {
             float acc[V];
 #pragma unroll
             for (int e = 0; e < V; ++e) acc[e] = 0.f;
@@ -62,7 +66,7 @@ pool_kernel(Geo g, const T* __restrict__ q, const T* __restrict__ k, float* __re
             for (int e = 0; e < V; ++e) r[e] = acc[e];
         }
         __syncthreads();
-        const int width = min(per_round, chunks - c0) * V;
+        const int width = min(per_round, cend - c0) * V;
         for (int e = threadIdx.x; e < width; e += kPoolThreads) {
             float s = 0.f;
             for (int gg = 0; gg < ngroups; ++gg) s += red[(size_t)gg * per_round * V + e];
@@ -83,9 +87,8 @@ cudaError_t launch_pool(const Geo& g, bsa_dtype dt, const void* q, const void* k
                         float* pk, cudaStream_t st) {
     const int V = dt == BSA_BF16 ? 8 : 4;
     const int chunks = g.H * g.d / V;
-    const int per_round = chunks < kPoolThreads ? chunks : kPoolThreads;
-    const size_t smem = (size_t)(kPoolThreads / per_round) * per_round * V * sizeof(float);
-    const dim3 grid(g.B, 2);
+    const size_t smem = (size_t)kPoolThreads * V * sizeof(float);   // ngroups x per_round <= 256 chunks
+    const dim3 grid(g.B, 2, (chunks + kChunksPerCta - 1) / kChunksPerCta);
     if (dt == BSA_BF16) {
         pool_kernel<__nv_bfloat16><<<grid, kPoolThreads, smem, st>>>(
             g, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), pq, pk);
