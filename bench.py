@@ -145,7 +145,7 @@ def step_calls(L, q, k, v, path: str):
     """The library calls of one layer, as (stage name, callable, our kernel launches)."""
     from view_transformers_b200 import _lib
     import torch
-    b = L.buf
+    b = L.buf if path == "fused" else L.partials()
     sp = torch.cuda.current_stream().cuda_stream
     status = b.status.data_ptr()
     lay = L.layout

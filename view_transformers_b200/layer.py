@@ -1,6 +1,8 @@
 """Runs one block-sparse global-attention layer through the C ABI.
 
-Torch provides the device buffers and the stream; each step is one library call:
+Torch provides the device buffers and the stream; each step is one library call.
+forward() on a bf16 layer: pack + pool -> predict mask -> special queries -> fused patch
+rows. The step-by-step path (predict(), attend(); f32 layers, or fused=False):
   pool -> predict mask -> pack -> special dense -> block-sparse attention -> merge.
 """
 from __future__ import annotations
@@ -22,12 +24,13 @@ class Buffers:
     kv_idx: torch.Tensor
     kv_cnt: torch.Tensor
     workspace: torch.Tensor
-    o_pp: torch.Tensor
-    lse_pp: torch.Tensor
-    o_ps: torch.Tensor
-    lse_ps: torch.Tensor
     out: torch.Tensor
     status: torch.Tensor
+    # fp32 partial results of the step-by-step path, allocated on its first use
+    o_pp: torch.Tensor | None = None
+    lse_pp: torch.Tensor | None = None
+    o_ps: torch.Tensor | None = None
+    lse_ps: torch.Tensor | None = None
 
 
 class BlockSparseLayer:
@@ -55,10 +58,6 @@ class BlockSparseLayer:
             kv_cnt=torch.empty((H, B), dtype=torch.int32, device=dev),
             # 1024-byte alignment for the TMA tiles: over-allocate and offset
             workspace=torch.empty(max(self.ws_bytes, 1) + 1024, dtype=torch.uint8, device=dev),
-            o_pp=torch.empty((self.Np, H, d), dtype=torch.float32, device=dev),
-            lse_pp=torch.empty((H, self.Np), dtype=torch.float32, device=dev),
-            o_ps=torch.empty((self.Np, H, d), dtype=torch.float32, device=dev),
-            lse_ps=torch.empty((H, self.Np), dtype=torch.float32, device=dev),
             out=torch.empty((self.N, H, d), dtype=_TORCH_DTYPE[dtype], device=dev),
             status=torch.zeros(1, dtype=torch.int32, device=dev),
         )
@@ -80,10 +79,21 @@ class BlockSparseLayer:
                               self.head_density, b.mask_bits.data_ptr(), b.kv_idx.data_ptr(),
                               b.kv_cnt.data_ptr(), b.status.data_ptr(), st)
 
+    def partials(self) -> Buffers:
+        """The layer's buffers, with the fp32 partials of the step-by-step path allocated."""
+        b = self.buf
+        if b.o_pp is None:
+            H, d, dev = self.H, self.d, self.device
+            b.o_pp = torch.empty((self.Np, H, d), dtype=torch.float32, device=dev)
+            b.lse_pp = torch.empty((H, self.Np), dtype=torch.float32, device=dev)
+            b.o_ps = torch.empty((self.Np, H, d), dtype=torch.float32, device=dev)
+            b.lse_ps = torch.empty((H, self.Np), dtype=torch.float32, device=dev)
+        return b
+
     def attend(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, stream: int | None = None,
                out: torch.Tensor | None = None) -> torch.Tensor:
         st = self._stream(stream)
-        b = self.buf
+        b = self.partials()
         o = self._out(out)
         qp, kp, vp = q.data_ptr(), k.data_ptr(), v.data_ptr()
         _lib.bsa_pack_qkv(self.layout, qp, kp, vp, self.ws_ptr, self.ws_bytes, b.status.data_ptr(), st)
