@@ -12,8 +12,8 @@
 // consecutive blocks of one dimension per load straight from L2; each lane accumulates
 // one block x 8 rows (8 independent FMA chains) with the query values of a dimension
 // broadcast from shared memory (one shared-memory wavefront feeds 4 FMAs per lane). The
-// small work items keep all 16 warps busy and the kernel within 64 registers, so two
-// CTAs share an SM.
+// kernel stays within 64 registers and about 46 KB of shared memory at B = 608, so four
+// 8-warp CTAs share an SM and cover each other's barrier between the two phases.
 //
 // Selection: instead of sorting a row, a select over the fp32 scores in three steps:
 //   - one pass counts the row into 256 equal-width score buckets over [min, max] (with
@@ -34,7 +34,7 @@
 namespace bsa {
 namespace {
 
-constexpr int kMaxWarps = 16;
+constexpr int kWarps = 8;         // per CTA; one query-block row each
 constexpr int kRadix = 256;
 constexpr int kDim = 64;
 
@@ -387,7 +387,7 @@ __device__ void select_row(const float* s, int B, int h, int i, int k, double ta
 
 // R query-block rows i0 .. i0+R-1 of head h per CTA.
 template <int R>
-__global__ void __launch_bounds__(32 * kMaxWarps, 2)
+__global__ void __launch_bounds__(64 * kWarps, 2)
 mask_kernel(Geo g, MaskParams mp, const float* __restrict__ pq, const float* __restrict__ pk,
             uint32_t* __restrict__ mask_bits, uint16_t* __restrict__ kv_idx,
             int32_t* __restrict__ kv_cnt, int32_t* status) {
@@ -496,13 +496,12 @@ cudaError_t launch_rows(const Geo& g, int W, const MaskParams& mp, const float* 
 cudaError_t launch_mask(const Geo& g, const MaskParams& mp, const float* pq, const float* pk,
                         uint32_t* mask_bits, uint16_t* kv_idx, int32_t* kv_cnt,
                         int32_t* status, cudaStream_t st) {
-    // 16 warps: the selection is a chain of dependent warp-wide steps per row, so it runs
-    // best with one row per warp and many rows in flight
-    const int W = kMaxWarps;
+    // 8 rows on 8 warps: one row per warp in the selection (a chain of dependent warp-wide
+    // steps), and small CTAs so that several share an SM and cover each other's barrier
+    // With long rows only one CTA fits on an SM: 16 warps then keep the score pass busier.
+    const int W = mask_smem<8>(g.B, kWarps) <= 113 * 1024 ? kWarps : 2 * kWarps;
     // the most rows per CTA whose score rows fit in shared memory
     const size_t limit = 227 * 1024;
-    if (mask_smem<16>(g.B, W) <= limit)
-        return launch_rows<16>(g, W, mp, pq, pk, mask_bits, kv_idx, kv_cnt, status, st);
     if (mask_smem<8>(g.B, W) <= limit)
         return launch_rows<8>(g, W, mp, pq, pk, mask_bits, kv_idx, kv_cnt, status, st);
     if (mask_smem<4>(g.B, W) <= limit)
