@@ -104,6 +104,7 @@ struct Ctl {
     uint32_t tmem_base;
     int n_tiles;
     int abort;
+    int head;
 };
 
 template <int BKV>
@@ -200,8 +201,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tmem_relinquish();
     }
     if (kUnion) {
+        // Heads in descending order of kept work (the kept-block counts of three query-block
+        // rows): CTAs of the heaviest heads start first, so the last wave holds light ones.
+        // Consecutive CTAs keep sharing a head (its keys stay hot in L2).
+        if (warp == 0) {
+            const bool sortable = g.H <= 32;
+            int w = -1;
+            if (sortable && lane < g.H) {
+                const int32_t* c = prm.kv_cnt + (size_t)lane * g.B;
+                w = min(c[0], g.B) + min(c[g.B / 2], g.B) + min(c[g.B - 1], g.B);
+            }
+            int r = 0;
+            for (int u = 0; u < 32; ++u) {
+                const int wu = __shfl_sync(0xffffffffu, w, u);
+                if (u < g.H && (wu > w || (wu == w && u < lane))) ++r;
+            }
+            const unsigned m = __ballot_sync(0xffffffffu, sortable && lane < g.H && r == h);
+            if (lane == 0) ctl.head = m ? __ffs(m) - 1 : h;
+        }
         for (int x = threadIdx.x; x < QB * words; x += kThreads) bits[x] = 0u;
         __syncthreads();
+        h = ctl.head;
         for (int qb = 0; qb < QB; ++qb) {
             const int i = tq * QB + qb;
             if (i >= g.B) break;
