@@ -99,12 +99,72 @@ struct Ctl {
     uint64_t o_done;
     uint64_t o_final;
     uint64_t drain;
-    int meta_nvalid[NS];
+    int meta_nvalid[NS];     // tile extents for the softmax when it does not compute them
     uint32_t meta_member[NS];
     uint32_t tmem_base;
     int n_tiles;
     int abort;
     int head;
+};
+
+// The key tiles of one CTA, in order: one key range of special and patch tiles
+// (MODE_SPECIAL_ALL), every special tile (MODE_PATCH_SPECIAL), or, for the fused and sparse
+// modes, the special tiles (fused only) followed by the kept blocks of the CTA's query blocks
+// (the union of their masks, ascending). The producer and every softmax warp run their own
+// copy, so a softmax warp learns a tile's extent and membership without a barrier.
+template <int MODE, int BKV>
+struct TileWalk {
+    static constexpr int QB = 128 / BKV;
+    struct Tile {
+        int row0;          // first packed row of the tile
+        int nvalid;        // rows of the tile that hold keys
+        uint32_t member;   // bit qb: query block qb of the tile kept this key block
+        bool special;      // tile of special keys
+    };
+    const uint32_t* bits;
+    int words;
+    int w = 0;
+    uint32_t cur = 0u;
+
+    __device__ __forceinline__ TileWalk(const uint32_t* b, int nw) : bits(b), words(nw) {
+        if ((MODE == MODE_SPARSE || MODE == MODE_FUSED) && nw > 0)
+            for (int qb = 0; qb < QB; ++qb) cur |= bits[qb * nw];
+    }
+
+    // Tile u (called for u = 0, 1, ... in order). False only if the union has no further
+    // block, which cannot happen for u below the CTA's tile count.
+    __device__ __forceinline__ bool next(int u, const Geo& g, const PackedLayout& pl, int h, int sp_tiles,
+                                         int t_begin, Tile& t) {
+        t.member = (1u << QB) - 1u;
+        if (MODE == MODE_SPECIAL_ALL) {
+            const int x = t_begin + u;
+            t.special = x < sp_tiles;
+            const int base = t.special ? x * 128 : (x - sp_tiles) * 128;
+            t.row0 = (t.special ? h * pl.ns_pad : h * pl.np_pad) + base;
+            t.nvalid = min(128, (t.special ? g.Ns : g.Np) - base);
+            return true;
+        }
+        if (MODE == MODE_PATCH_SPECIAL || (MODE == MODE_FUSED && u < sp_tiles)) {
+            t.special = true;
+            t.row0 = h * pl.ns_pad + u * BKV;
+            t.nvalid = min(BKV, g.Ns - u * BKV);
+            return true;
+        }
+        t.special = false;
+        while (cur == 0u && w + 1 < words) {
+            ++w;
+            for (int qb = 0; qb < QB; ++qb) cur |= bits[qb * words + w];
+        }
+        if (cur == 0u) return false;
+        const int bit = __ffs(cur) - 1;
+        cur &= cur - 1u;
+        const int j = w * 32 + bit;
+        t.member = 0u;
+        for (int qb = 0; qb < QB; ++qb) t.member |= ((bits[qb * words + w] >> bit) & 1u) << qb;
+        t.row0 = h * pl.np_pad + j * BKV;
+        t.nvalid = min(BKV, g.Np - j * BKV);
+        return true;
+    }
 };
 
 template <int BKV>
@@ -135,8 +195,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     using C = Cfg<BKV>;
     constexpr int NS = C::NS;
     constexpr int QB = C::QB;
-    constexpr uint32_t kAll = (1u << QB) - 1u;
     constexpr bool kUnion = MODE == MODE_SPARSE || MODE == MODE_FUSED;   // walks kept blocks
+    // With one query block per tile (b = 128) a softmax warp computes each tile's extent
+    // itself; with two (b = 64) it reads what the producer stored for the stage, after the
+    // stage's kv_full barrier (walking the union mask per warp costs more than that wait).
+    constexpr bool kLocalTiles = QB == 1;
     extern __shared__ __align__(1024) uint8_t smem[];
     Ctl<NS>& ctl = *reinterpret_cast<Ctl<NS>*>(smem + C::kOffCtl);
     uint32_t* bits = reinterpret_cast<uint32_t*>(smem + C::kOffCtl + (sizeof(Ctl<NS>) + 15) / 16 * 16);
@@ -262,48 +325,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const int q_row0 = MODE == MODE_SPECIAL_ALL ? h * pl.ns_pad + tq * 128 : h * pl.np_pad + tq * 128;
             mbar_arrive_expect_tx(&ctl.q_full, 128 * 128);
             tma_load_2d(smem + C::kOffQ, &tm_q, &ctl.q_full, 0, q_row0);
-            int w = 0;
-            uint32_t cur = 0;
-            if (kUnion && words > 0)
-                for (int qb = 0; qb < QB; ++qb) cur |= bits[qb * words];
+            TileWalk<MODE, BKV> walk(bits, words);
             for (int u = 0; u < n; ++u) {
                 const int stage = u % NS;
                 if (u >= NS && !mbar_wait(&ctl.kv_empty[stage], ((u / NS) - 1) & 1, abort, prm.status)) break;
-                int row0, nvalid;
-                uint32_t member = kAll;
-                bool special;
-                if (MODE == MODE_SPECIAL_ALL) {
-                    const int t = t_begin + u;
-                    special = t < sp_tiles;
-                    const int base = special ? t * 128 : (t - sp_tiles) * 128;
-                    row0 = (special ? h * pl.ns_pad : h * pl.np_pad) + base;
-                    nvalid = min(128, (special ? g.Ns : g.Np) - base);
-                } else if (MODE == MODE_PATCH_SPECIAL || (MODE == MODE_FUSED && u < sp_tiles)) {
-                    special = true;
-                    row0 = h * pl.ns_pad + u * BKV;
-                    nvalid = min(BKV, g.Ns - u * BKV);
-                } else {
-                    special = false;
-                    while (cur == 0u && w + 1 < words) {
-                        ++w;
-                        for (int qb = 0; qb < QB; ++qb) cur |= bits[qb * words + w];
-                    }
-                    if (cur == 0u) break;
-                    const int bit = __ffs(cur) - 1;
-                    cur &= cur - 1u;
-                    const int j = w * 32 + bit;
-                    member = 0u;
-                    for (int qb = 0; qb < QB; ++qb) member |= ((bits[qb * words + w] >> bit) & 1u) << qb;
-                    row0 = h * pl.np_pad + j * BKV;
-                    nvalid = min(BKV, g.Np - j * BKV);
+                typename TileWalk<MODE, BKV>::Tile t;
+                if (!walk.next(u, g, pl, h, sp_tiles, t_begin, t)) break;
+                if (!kLocalTiles) {
+                    ctl.meta_nvalid[stage] = t.nvalid;
+                    ctl.meta_member[stage] = t.member;
                 }
-                ctl.meta_nvalid[stage] = nvalid;
-                ctl.meta_member[stage] = member;
                 mbar_arrive_expect_tx(&ctl.kv_full[stage], 2 * C::kTileBytes);
-                tma_load_2d(smem + C::kOffK + stage * C::kTileBytes, special ? &tm_ka : &tm_kb, &ctl.kv_full[stage],
-                            0, row0);
-                tma_load_2d(smem + C::kOffV + stage * C::kTileBytes, special ? &tm_va : &tm_vb, &ctl.kv_full[stage],
-                            0, row0);
+                tma_load_2d(smem + C::kOffK + stage * C::kTileBytes, t.special ? &tm_ka : &tm_kb,
+                            &ctl.kv_full[stage], 0, t.row0);
+                tma_load_2d(smem + C::kOffV + stage * C::kTileBytes, t.special ? &tm_va : &tm_vb,
+                            &ctl.kv_full[stage], 0, t.row0);
                 issued = u + 1;
             }
             if (n == 0) drain_wait(&ctl.q_full, 0, prm.status);   // no MMA will consume Q
@@ -354,11 +390,30 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         float m_ref = -INFINITY;
         float l = 0.f;
         bool ok = true;
+        // Tile extents as the producer's walk yields them. With one query block per tile the
+        // kept blocks come in ascending order and each is a member, so only the last tile can
+        // be the ragged last patch block; the special-key modes are plain arithmetic.
+        const bool tail_kept = kLocalTiles && kUnion && g.B > 0 &&
+                               ((bits[(g.B - 1) >> 5] >> ((g.B - 1) & 31)) & 1u) != 0u;
+        const int tail_rows = g.Np - (g.B - 1) * BKV;
+        TileWalk<MODE, BKV> walk(bits, 0);   // arithmetic modes only: no mask state
         for (int u = 0; u < n; ++u) {
-            const int stage = u % NS;
-            if (!warp_wait(&ctl.kv_full[stage], (u / NS) & 1, abort, prm.status)) { ok = false; break; }
-            const int nvalid = ctl.meta_nvalid[stage];
-            const bool member = ((ctl.meta_member[stage] >> row_qb) & 1u) != 0u;
+            int nvalid;
+            uint32_t members = 1u;
+            if (kLocalTiles && kUnion) {
+                nvalid = MODE == MODE_FUSED && u < sp_tiles ? min(BKV, g.Ns - u * BKV)
+                       : (u == n - 1 && tail_kept) ? tail_rows : BKV;
+            } else if (kLocalTiles) {
+                typename TileWalk<MODE, BKV>::Tile t;
+                walk.next(u, g, pl, h, sp_tiles, t_begin, t);
+                nvalid = t.nvalid;
+            } else {
+                const int stage = u % NS;
+                if (!warp_wait(&ctl.kv_full[stage], (u / NS) & 1, abort, prm.status)) { ok = false; break; }
+                nvalid = ctl.meta_nvalid[stage];
+                members = ctl.meta_member[stage];
+            }
+            const bool member = ((members >> row_qb) & 1u) != 0u;
             const bool full = member && nvalid == BKV;
             if (!warp_wait(&ctl.s_full, u & 1, abort, prm.status)) { ok = false; break; }
             tc_fence_after();
@@ -407,7 +462,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                                 scale2, shift2);
                     const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
                     r2[i & 3] = __fadd2_rn(r2[i & 3], pr);
-                    s[i] = pack_half2(pr.x, pr.y);   // pair i lands in s[i] after s[2i], s[2i+1] were read
+                    s[i] = pack_half2(pr.x, pr.y);
                 }
                 rs = ((r2[0].x + r2[0].y) + (r2[1].x + r2[1].y)) + ((r2[2].x + r2[2].y) + (r2[3].x + r2[3].y));
             } else {
@@ -418,8 +473,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     const float p1 =
                         member && c + 1 < nvalid ? ex2_approx(fmaf(__uint_as_float(s[c + 1]), kScaleLog2, -m_ref)) : 0.f;
                     rs += p0 + p1;
-                    const __half2 hp = __floats2half2_rn(p0, p1);
-                    s[c / 2] = *reinterpret_cast<const uint32_t*>(&hp);
+                    s[c / 2] = pack_half2(p0, p1);
                 }
             }
             l = l * factor + rs;
@@ -429,7 +483,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 break;
             }
             tc_fence_after();
-            if (__any_sync(0xffffffffu, corr)) {
+            if (__any_sync(0xffffffffu, corr)) {   // lazy rescale of O, before P.V of this tile
 #pragma unroll
                 for (int a = 0; a < 2; ++a) {
                     uint32_t o[32];
