@@ -150,6 +150,9 @@ EDGE = [
     configs.Workload("tail1_b128", 1, 129, 5, 2, 64, 128, 0.5, 0.0, "bf16", "five_percent"),
     configs.Workload("b33_blocks", 3, 703, 5, 2, 64, 64, 0.6, 0.0, "bf16", "five_percent"),
     configs.Workload("f32_tail1", 3, 11, 4, 2, 64, 16, 0.5, 0.3, "f32", "tiny"),
+    # an odd number of (query tile, head) items at b = 128 (the fused kernel pairs them), with
+    # uneven kept counts between the rows of a pair
+    configs.Workload("odd_items_b128", 3, 777, 5, 3, 64, 128, 0.5, 0.5, "bf16", "five_percent"),
 ]
 
 
