@@ -385,7 +385,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-budget", type=float, default=3.0, help="seconds of oracle work per reference step")
     ap.add_argument("--dense-steps", type=int, default=3)
-    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--frames", type=int, default=None,
                     help="override the workload's frame count (smaller cases for profiling)")
     ap.add_argument("--path", default=None, choices=["fused", "five"],

@@ -27,8 +27,10 @@
 // kept blocks, and each row ignores the key blocks its own query block did not keep.
 //
 // Barrier protocol (u = tile index of the CTA). A parity wait only tells apart phases
-// within one of the barrier's current phase; every wait below has that property:
-//   kv_full[s]/kv_empty[s]  TMA ring; the producer refills a stage after P.V of its tile;
+// within one phase of the barrier's current one; every wait below has that property:
+//   kv_full[s]/kv_empty[s]  TMA ring; the producer refills a stage after P.V of its tile.
+//            For b = 64 the softmax also waits on kv_full to read the tile's extent and
+//            membership, which the producer stores per stage;
 //   s_full   QK^T of tile u done (commit; also implies every earlier MMA is done);
 //   s_free   all 4 softmax warps have S_u in registers (count 4) -> QK^T of tile u+1;
 //   p_full   all 4 softmax warps wrote P_u (count 4) -> P.V of tile u;
