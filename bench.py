@@ -115,6 +115,19 @@ def measured_traffic(w, path):
 
 
 
+def xu_roofline(f_kernel, kernel_ms, w, clocks) -> dict:
+    """The attention kernel's other bound: one ex2 per computed score entry (f_kernel / 4d
+    entries) on the special-function unit, 16 ex2 per clock per SM (measured on this B200 by a
+    back-to-back ex2.approx.f32 microbenchmark), 148 SMs, at the median SM clock sampled during
+    the timed region."""
+    entries = f_kernel / (4.0 * w.head_dim)
+    achieved = entries / (kernel_ms * 1e-3)
+    mhz = clocks.get("sm_mhz") or 1965.0
+    peak = 16.0 * 148 * mhz * 1e6
+    return {"bound": "xu", "achieved": achieved, "peak": peak, "unit": "ex2/s", "frac": achieved / peak,
+            "peak_kind": "16 ex2/clock/SM x 148 SMs x sampled SM clock"}
+
+
 def sparse_flops(kv_cnt, kv_idx, w) -> float:
     """4 d sum_h sum_(i, j kept) |I_i| |J_j| over patch query/key blocks."""
     B, b, Np = w.n_blocks, w.block, w.n_patch
@@ -497,7 +510,8 @@ def main():
                      "frac_of_burst": achieved / tf_burst, "frac_of_nominal_2250": achieved / 2250.0,
                      "flops_per_launch": f_kernel, "launch_ms": sparse_ms,
                      "launch_ms_alone": stage_ms["sparse"], "traffic": measured_traffic(w, path),
-                     "traffic_unit": "bytes per launch (ncu dram read+write, scaled by patch tokens x heads)"},
+                     "traffic_unit": "bytes per launch (ncu dram read+write, scaled by patch tokens x heads)",
+                     "xu": xu_roofline(f_kernel, sparse_ms, w, clocks)},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": args.e2e_steps,
                 "copies": "pinned host buffers; inputs of step s+1 and output of step s-1 copied on "
