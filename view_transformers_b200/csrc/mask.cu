@@ -385,33 +385,38 @@ __device__ void select_row(const float* s, int B, int h, int i, int k, double ta
     }
 }
 
-// R query-block rows i0 .. i0+R-1 of head h per CTA.
+// Row stride of the transposed query block in shared memory: 16-byte aligned rows.
 template <int R>
-__global__ void __launch_bounds__(64 * kWarps, 2)
+__host__ __device__ constexpr int q_stride() { return (R + 3) / 4 * 4; }
+
+// R query-block rows i0 .. i0+R-1 of head h per CTA, on W warps (at most 16; MINB CTAs per
+// SM in the launch bounds).
+template <int R, int W, int MINB>
+__global__ void __launch_bounds__(32 * W, MINB)
 mask_kernel(Geo g, MaskParams mp, const float* __restrict__ pq, const float* __restrict__ pk,
             uint32_t* __restrict__ mask_bits, uint16_t* __restrict__ kv_idx,
             int32_t* __restrict__ kv_cnt, int32_t* status) {
     extern __shared__ __align__(16) unsigned char smem[];
-    const int W = blockDim.x / 32;
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
     const int h = blockIdx.y;
     const int B = g.B;
     const int i0 = blockIdx.x * R;
 
-    float* qT = reinterpret_cast<float*>(smem);                        // [d][R]
-    WarpHist* hists = reinterpret_cast<WarpHist*>(qT + kDim * R);      // [W]
+    constexpr int QS = q_stride<R>();
+    float* qT = reinterpret_cast<float*>(smem);                        // [d][QS]
+    WarpHist* hists = reinterpret_cast<WarpHist*>(qT + kDim * QS);     // [W]
     float* sc = reinterpret_cast<float*>(hists + W);                   // [R][B]
 
     for (int x = threadIdx.x; x < R * kDim; x += blockDim.x) {
         const int r = x / kDim, d = x % kDim;
-        qT[d * R + r] = i0 + r < B ? pq[((size_t)h * B + i0 + r) * kDim + d] : 0.f;
+        qT[d * QS + r] = i0 + r < B ? pq[((size_t)h * B + i0 + r) * kDim + d] : 0.f;
     }
     __syncthreads();
 
     // ---- pooled scores: work items of 32 blocks (one per lane) x RG rows, round-robin over
     // the warps (consecutive warps take consecutive block chunks)
-    constexpr int RG = R < 8 ? R : 8;
+    constexpr int RG = R <= 9 ? R : 8;   // rows per work item; R is a multiple of RG
     const float* pk_h = pk + (size_t)h * kDim * B;
     const float scale = 0.125f;   // 1 / sqrt(64)
     const int nchunk = (B + 31) / 32;
@@ -437,19 +442,21 @@ mask_kernel(Geo g, MaskParams mp, const float* __restrict__ pq, const float* __r
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const float* qd = qT + (d0 + u) * R + rg * RG;
+                const float* qd = qT + (d0 + u) * QS + rg * RG;
 #pragma unroll
-                for (int r4 = 0; r4 < RG; r4 += (RG >= 4 ? 4 : RG)) {
+                for (int r4 = 0; r4 < RG; r4 += 4) {
+                    constexpr int kAll4 = RG >= 4;
                     float qv[4];
-                    if constexpr (RG >= 4) {
+                    if (kAll4 && r4 + 4 <= RG) {   // 16-byte aligned: QS and RG (1, 2, 4, 8) keep it
                         const float4 t = *reinterpret_cast<const float4*>(qd + r4);
                         qv[0] = t.x; qv[1] = t.y; qv[2] = t.z; qv[3] = t.w;
                     } else {
 #pragma unroll
-                        for (int e = 0; e < RG; ++e) qv[e] = qd[e];
+                        for (int e = 0; e < 4; ++e) qv[e] = r4 + e < RG ? qd[r4 + e] : 0.f;
                     }
 #pragma unroll
-                    for (int e = 0; e < (RG >= 4 ? 4 : RG); ++e) a[r4 + e] = fmaf(qv[e], kc[u], a[r4 + e]);
+                    for (int e = 0; e < 4; ++e)
+                        if (r4 + e < RG) a[r4 + e] = fmaf(qv[e], kc[u], a[r4 + e]);
                 }
             }
             if (d0 + 8 < kDim) {
@@ -475,19 +482,19 @@ mask_kernel(Geo g, MaskParams mp, const float* __restrict__ pq, const float* __r
 
 template <int R>
 size_t mask_smem(int B, int W) {
-    return (size_t)kDim * R * 4 + sizeof(WarpHist) * W + (size_t)R * B * 4;
+    return (size_t)kDim * q_stride<R>() * 4 + sizeof(WarpHist) * W + (size_t)R * B * 4;
 }
 
-template <int R>
-cudaError_t launch_rows(const Geo& g, int W, const MaskParams& mp, const float* pq, const float* pk,
+template <int R, int W, int MINB>
+cudaError_t launch_rows(const Geo& g, const MaskParams& mp, const float* pq, const float* pk,
                         uint32_t* mask_bits, uint16_t* kv_idx, int32_t* kv_cnt, int32_t* status,
                         cudaStream_t st) {
     const size_t smem = mask_smem<R>(g.B, W);
-    cudaError_t e = cudaFuncSetAttribute(mask_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    auto kern = mask_kernel<R, W, MINB>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const dim3 grid((g.B + R - 1) / R, g.H);
-    mask_kernel<R><<<grid, 32 * W, smem, st>>>(g, mp, pq, pk, mask_bits, kv_idx, kv_cnt, status);
+    kern<<<grid, 32 * W, smem, st>>>(g, mp, pq, pk, mask_bits, kv_idx, kv_cnt, status);
     return cudaGetLastError();
 }
 
@@ -497,17 +504,27 @@ cudaError_t launch_mask(const Geo& g, const MaskParams& mp, const float* pq, con
                         uint32_t* mask_bits, uint16_t* kv_idx, int32_t* kv_cnt,
                         int32_t* status, cudaStream_t st) {
     // 8 rows on 8 warps: one row per warp in the selection (a chain of dependent warp-wide
-    // steps), and small CTAs so that several share an SM and cover each other's barrier
+    // steps), and small CTAs so that four share an SM (64 registers per thread) and cover
+    // each other's barrier. When the rows leave a small last round of CTAs (e.g. 2.05 rounds
+    // of 4 x 148 CTAs at 100 frames), 9 rows on 9 warps (at most 56 registers, so that four
+    // CTAs still fit) finish in one round fewer.
     // With long rows only one CTA fits on an SM: 16 warps then keep the score pass busier.
-    const int W = mask_smem<8>(g.B, kWarps) <= 113 * 1024 ? kWarps : 2 * kWarps;
+    const size_t per_sm = 228 * 1024;
+    const int slots = num_sms() * 4;
+    const long long ctas8 = (long long)((g.B + 7) / 8) * g.H, ctas9 = (long long)((g.B + 8) / 9) * g.H;
+    if (4 * (mask_smem<9>(g.B, 9) + 1024) <= per_sm && (ctas9 + slots - 1) / slots < (ctas8 + slots - 1) / slots)
+        return launch_rows<9, 9, 4>(g, mp, pq, pk, mask_bits, kv_idx, kv_cnt, status, st);
+    const bool small = mask_smem<8>(g.B, kWarps) <= 113 * 1024;
     // the most rows per CTA whose score rows fit in shared memory
     const size_t limit = 227 * 1024;
-    if (mask_smem<8>(g.B, W) <= limit)
-        return launch_rows<8>(g, W, mp, pq, pk, mask_bits, kv_idx, kv_cnt, status, st);
-    if (mask_smem<4>(g.B, W) <= limit)
-        return launch_rows<4>(g, W, mp, pq, pk, mask_bits, kv_idx, kv_cnt, status, st);
-    if (mask_smem<1>(g.B, W) <= limit)
-        return launch_rows<1>(g, W, mp, pq, pk, mask_bits, kv_idx, kv_cnt, status, st);
+    // (the launch bounds keep every variant within 64 registers per thread)
+    if (small) return launch_rows<8, kWarps, 4>(g, mp, pq, pk, mask_bits, kv_idx, kv_cnt, status, st);
+    if (mask_smem<8>(g.B, 2 * kWarps) <= limit)
+        return launch_rows<8, 2 * kWarps, 2>(g, mp, pq, pk, mask_bits, kv_idx, kv_cnt, status, st);
+    if (mask_smem<4>(g.B, 2 * kWarps) <= limit)
+        return launch_rows<4, 2 * kWarps, 2>(g, mp, pq, pk, mask_bits, kv_idx, kv_cnt, status, st);
+    if (mask_smem<1>(g.B, 2 * kWarps) <= limit)
+        return launch_rows<1, 2 * kWarps, 2>(g, mp, pq, pk, mask_bits, kv_idx, kv_cnt, status, st);
     return cudaErrorInvalidValue;
 }
 
