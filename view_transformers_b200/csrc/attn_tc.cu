@@ -24,7 +24,10 @@
 //               p = 2^(s log2(e)/sqrt(d) - m) in fp32, P rounded to fp16 into TMEM,
 //               then the epilogue O / l and the log-sum-exp.
 // For b = 64 a 128-row query tile holds two query blocks; it walks the union of their
-// kept blocks, and each row ignores the key blocks its own query block did not keep.
+// kept blocks, two per 128-key tile. The softmax computes every column of a tile whose kept
+// blocks are whole and then drops, by selects, the block a row's query block did not keep
+// (from the row max, the row sum and P); only tiles with a ragged kept block go column by
+// column.
 //
 // Barrier protocol (u = tile index of the CTA). A parity wait only tells apart phases
 // within one phase of the barrier's current one; every wait below has that property:
@@ -79,11 +82,15 @@ struct TcParams {
     int q_tiles;   // query tiles per head
 };
 
+// BKV is the block size b (64 or 128). Query and key tiles are always 128 rows: a key tile
+// holds one block of 128 keys or two kept blocks of 64 (not necessarily adjacent), so that
+// QK^T runs at N = 128 and each tile's fixed costs cover 128 keys.
 template <int BKV>
 struct Cfg {
-    static constexpr int NS = BKV == 128 ? 3 : 6;   // K/V stages
+    static constexpr int NS = 3;                    // K/V stages
     static constexpr int QB = 128 / BKV;            // query blocks per 128-row query tile
-    static constexpr uint32_t kTileBytes = BKV * 128;
+    static constexpr int KB = 128 / BKV;            // key blocks per 128-key tile
+    static constexpr uint32_t kTileBytes = 128 * 128;
     static constexpr uint32_t kOffQ = 0;
     static constexpr uint32_t kOffK = kOffQ + 128 * 128;
     static constexpr uint32_t kOffV = kOffK + NS * kTileBytes;
@@ -101,8 +108,8 @@ struct Ctl {
     uint64_t o_done;
     uint64_t o_final;
     uint64_t drain;
-    int meta_nvalid[NS];     // tile extents for the softmax when it does not compute them
-    uint32_t meta_member[NS];
+    int meta_nvalid[NS];     // tile extents for the softmax when it does not compute them: row
+    uint32_t meta_member[NS];   // counts of the key blocks (8 bits each) and their membership bits
     uint32_t tmem_base;
     int n_tiles;
     int abort;
@@ -112,59 +119,71 @@ struct Ctl {
 // The key tiles of one CTA, in order: one key range of special and patch tiles
 // (MODE_SPECIAL_ALL), every special tile (MODE_PATCH_SPECIAL), or, for the fused and sparse
 // modes, the special tiles (fused only) followed by the kept blocks of the CTA's query blocks
-// (the union of their masks, ascending). The producer and every softmax warp run their own
-// copy, so a softmax warp learns a tile's extent and membership without a barrier.
+// (the union of their masks, ascending), KB blocks per tile. The producer runs it, and for
+// b = 128 the softmax warps run the arithmetic part of their own copy, so they learn a tile's
+// extent without a barrier. A tile with fewer than KB kept blocks left loads its missing
+// block from a row past the end of the packed array, which reads zeros.
 template <int MODE, int BKV>
 struct TileWalk {
     static constexpr int QB = 128 / BKV;
+    static constexpr int KB = 128 / BKV;
     struct Tile {
-        int row0;          // first packed row of the tile
-        int nvalid;        // rows of the tile that hold keys
-        uint32_t member;   // bit qb: query block qb of the tile kept this key block
+        int row0[KB];      // first packed row of each key block
+        int nvalid[KB];    // rows of each key block that hold keys (0 for a missing block)
+        uint32_t member;   // bit k * QB + qb: query block qb of the tile kept key block k
         bool special;      // tile of special keys
     };
     const uint32_t* bits;
     int words;
     int w = 0;
     uint32_t cur = 0u;
-
     __device__ __forceinline__ TileWalk(const uint32_t* b, int nw) : bits(b), words(nw) {
         if ((MODE == MODE_SPARSE || MODE == MODE_FUSED) && nw > 0)
             for (int qb = 0; qb < QB; ++qb) cur |= bits[qb * nw];
     }
-
     // Tile u (called for u = 0, 1, ... in order). False only if the union has no further
     // block, which cannot happen for u below the CTA's tile count.
     __device__ __forceinline__ bool next(int u, const Geo& g, const PackedLayout& pl, int h, int sp_tiles,
                                          int t_begin, Tile& t) {
-        t.member = (1u << QB) - 1u;
+        t.member = (1u << (KB * QB)) - 1u;
         if (MODE == MODE_SPECIAL_ALL) {
             const int x = t_begin + u;
             t.special = x < sp_tiles;
             const int base = t.special ? x * 128 : (x - sp_tiles) * 128;
-            t.row0 = (t.special ? h * pl.ns_pad : h * pl.np_pad) + base;
-            t.nvalid = min(128, (t.special ? g.Ns : g.Np) - base);
+            t.row0[0] = (t.special ? h * pl.ns_pad : h * pl.np_pad) + base;
+            t.nvalid[0] = min(128, (t.special ? g.Ns : g.Np) - base);
             return true;
         }
         if (MODE == MODE_PATCH_SPECIAL || (MODE == MODE_FUSED && u < sp_tiles)) {
             t.special = true;
-            t.row0 = h * pl.ns_pad + u * BKV;
-            t.nvalid = min(BKV, g.Ns - u * BKV);
+#pragma unroll
+            for (int k = 0; k < KB; ++k) {
+                t.row0[k] = h * pl.ns_pad + u * 128 + k * BKV;
+                t.nvalid[k] = max(0, min(BKV, g.Ns - (u * 128 + k * BKV)));
+            }
             return true;
         }
         t.special = false;
-        while (cur == 0u && w + 1 < words) {
-            ++w;
-            for (int qb = 0; qb < QB; ++qb) cur |= bits[qb * words + w];
-        }
-        if (cur == 0u) return false;
-        const int bit = __ffs(cur) - 1;
-        cur &= cur - 1u;
-        const int j = w * 32 + bit;
         t.member = 0u;
-        for (int qb = 0; qb < QB; ++qb) t.member |= ((bits[qb * words + w] >> bit) & 1u) << qb;
-        t.row0 = h * pl.np_pad + j * BKV;
-        t.nvalid = min(BKV, g.Np - j * BKV);
+#pragma unroll
+        for (int k = 0; k < KB; ++k) {
+            while (cur == 0u && w + 1 < words) {
+                ++w;
+                for (int qb = 0; qb < QB; ++qb) cur |= bits[qb * words + w];
+            }
+            if (cur == 0u) {
+                if (k == 0) return false;
+                t.row0[k] = g.H * pl.np_pad;   // past the end: zeros
+                t.nvalid[k] = 0;
+                continue;
+            }
+            const int bit = __ffs(cur) - 1;
+            cur &= cur - 1u;
+            const int j = w * 32 + bit;
+            for (int qb = 0; qb < QB; ++qb) t.member |= ((bits[qb * words + w] >> bit) & 1u) << (k * QB + qb);
+            t.row0[k] = h * pl.np_pad + j * BKV;
+            t.nvalid[k] = min(BKV, g.Np - j * BKV);
+        }
         return true;
     }
 };
@@ -197,11 +216,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     using C = Cfg<BKV>;
     constexpr int NS = C::NS;
     constexpr int QB = C::QB;
+    constexpr int KB = C::KB;
     constexpr bool kUnion = MODE == MODE_SPARSE || MODE == MODE_FUSED;   // walks kept blocks
     // With one query block per tile (b = 128) a softmax warp computes each tile's extent
     // itself; with two (b = 64) it reads what the producer stored for the stage, after the
     // stage's kv_full barrier (walking the union mask per warp costs more than that wait).
-    constexpr bool kLocalTiles = QB == 1;
+    constexpr bool kLocalTiles = KB == 1;
     extern __shared__ __align__(1024) uint8_t smem[];
     Ctl<NS>& ctl = *reinterpret_cast<Ctl<NS>*>(smem + C::kOffCtl);
     uint32_t* bits = reinterpret_cast<uint32_t*>(smem + C::kOffCtl + (sizeof(Ctl<NS>) + 15) / 16 * 16);
@@ -230,7 +250,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         h = blockIdx.x / prm.q_tiles;
         tq = blockIdx.x - h * prm.q_tiles;
     }
-    const int sp_tiles = (g.Ns + BKV - 1) / BKV;   // special key tiles (BKV rows)
+    const int sp_tiles = (g.Ns + 127) / 128;       // special key tiles (128 rows)
     int t_begin = 0, t_end = 0;                    // MODE_SPECIAL_ALL key-tile range
     if (MODE == MODE_SPECIAL_ALL) {
         const int n_all = sp_tiles + pl.np_pad / 128;   // even split: sizes differ by at most one
@@ -315,8 +335,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ctl.tmem_base;
-    const int n = MODE == MODE_SPARSE ? ctl.n_tiles
-                : MODE == MODE_FUSED ? sp_tiles + ctl.n_tiles
+    const int kept_tiles = (ctl.n_tiles + KB - 1) / KB;   // KB kept blocks per tile
+    const int n = MODE == MODE_SPARSE ? kept_tiles
+                : MODE == MODE_FUSED ? sp_tiles + kept_tiles
                 : MODE == MODE_PATCH_SPECIAL ? sp_tiles
                 : t_end - t_begin;
     int issued = 0;   // K/V tiles whose loads the producer issued
@@ -334,14 +355,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 typename TileWalk<MODE, BKV>::Tile t;
                 if (!walk.next(u, g, pl, h, sp_tiles, t_begin, t)) break;
                 if (!kLocalTiles) {
-                    ctl.meta_nvalid[stage] = t.nvalid;
+                    int nv = 0;
+#pragma unroll
+                    for (int k = 0; k < KB; ++k) nv |= t.nvalid[k] << (8 * k);
+                    ctl.meta_nvalid[stage] = nv;
                     ctl.meta_member[stage] = t.member;
                 }
                 mbar_arrive_expect_tx(&ctl.kv_full[stage], 2 * C::kTileBytes);
-                tma_load_2d(smem + C::kOffK + stage * C::kTileBytes, t.special ? &tm_ka : &tm_kb,
-                            &ctl.kv_full[stage], 0, t.row0);
-                tma_load_2d(smem + C::kOffV + stage * C::kTileBytes, t.special ? &tm_va : &tm_vb,
-                            &ctl.kv_full[stage], 0, t.row0);
+#pragma unroll
+                for (int k = 0; k < KB; ++k) {   // block k fills rows [k * BKV, (k + 1) * BKV) of the stage
+                    const uint32_t off = stage * C::kTileBytes + (uint32_t)k * BKV * 128;
+                    tma_load_2d(smem + C::kOffK + off, t.special ? &tm_ka : &tm_kb, &ctl.kv_full[stage], 0,
+                                t.row0[k]);
+                    tma_load_2d(smem + C::kOffV + off, t.special ? &tm_va : &tm_vb, &ctl.kv_full[stage], 0,
+                                t.row0[k]);
+                }
                 issued = u + 1;
             }
             if (n == 0) drain_wait(&ctl.q_full, 0, prm.status);   // no MMA will consume Q
@@ -349,7 +377,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     } else if (warp == 1) {
         // ============================================================ MMA issuer
         if (lane == 0 && n > 0 && mbar_wait(&ctl.q_full, 0, abort, prm.status)) {
-            constexpr uint32_t idesc_qk = idesc_f16(128, BKV, 1u, false);
+            constexpr uint32_t idesc_qk = idesc_f16(128, 128, 1u, false);
             constexpr uint32_t idesc_pv = idesc_f16(128, 64, 0u, true);
             const uint32_t q_base = smem_u32(smem + C::kOffQ);
             auto issue_qk = [&](int u) -> bool {
@@ -375,7 +403,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const int stage = u % NS;
                 const uint32_t v_base = smem_u32(smem + C::kOffV + stage * C::kTileBytes);
 #pragma unroll
-                for (int ks = 0; ks < BKV / 16; ++ks)
+                for (int ks = 0; ks < 128 / 16; ++ks)
                     mma_ts(tmem + kColO, tmem + kColP + 8 * ks, sdesc_sw128(v_base + 2048 * ks, 0, 1024), idesc_pv,
                            (u > 0 || ks > 0) ? 1u : 0u);
                 mma_commit(&ctl.kv_empty[stage]);
@@ -399,35 +427,65 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                ((bits[(g.B - 1) >> 5] >> ((g.B - 1) & 31)) & 1u) != 0u;
         const int tail_rows = g.Np - (g.B - 1) * BKV;
         TileWalk<MODE, BKV> walk(bits, 0);   // arithmetic modes only: no mask state
+        constexpr int TC = 128;   // key columns per tile
         for (int u = 0; u < n; ++u) {
             int nvalid;
             uint32_t members = 1u;
+            int nv1 = 0;            // b = 64: rows of the tile's second key block
             if (kLocalTiles && kUnion) {
                 nvalid = MODE == MODE_FUSED && u < sp_tiles ? min(BKV, g.Ns - u * BKV)
                        : (u == n - 1 && tail_kept) ? tail_rows : BKV;
             } else if (kLocalTiles) {
                 typename TileWalk<MODE, BKV>::Tile t;
                 walk.next(u, g, pl, h, sp_tiles, t_begin, t);
-                nvalid = t.nvalid;
+                nvalid = t.nvalid[0];
             } else {
                 const int stage = u % NS;
                 if (!warp_wait(&ctl.kv_full[stage], (u / NS) & 1, abort, prm.status)) { ok = false; break; }
-                nvalid = ctl.meta_nvalid[stage];
+                const int packed = ctl.meta_nvalid[stage];
+                nvalid = packed & 0xff;
+                nv1 = (packed >> 8) & 0xff;
                 members = ctl.meta_member[stage];
             }
             const bool member = ((members >> row_qb) & 1u) != 0u;
-            const bool full = member && nvalid == BKV;
+            bool full = member && nvalid == BKV;
+            // b = 64: key block k of the tile is kept by this row's query block (mem1 for k = 1);
+            // a tile is ragged when a kept block has fewer than 64 keys
+            const bool mem1 = KB == 2 && ((members >> (QB + row_qb)) & 1u) != 0u;
+            const bool ragged = KB == 2 && ((member && nvalid < BKV) || (mem1 && nv1 < BKV));
+            if (KB == 2) full = !ragged;
             if (!warp_wait(&ctl.s_full, u & 1, abort, prm.status)) { ok = false; break; }
             tc_fence_after();
-            uint32_t s[BKV];
+            uint32_t s[TC];
 #pragma unroll
-            for (int c = 0; c < BKV / 32; ++c)
+            for (int c = 0; c < TC / 32; ++c)
                 tmem_ld32(lane_base + kColS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&s[32 * c]));
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&ctl.s_free);   // the next QK^T may overwrite S
             float mt = -INFINITY;
+            if constexpr (KB == 2) {
+                if (full) {   // both half maxima; a half this row's query block did not keep is dropped
+                    float acc[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc[i] = __uint_as_float(s[(i & 3) + (i >> 2) * 64]);
+#pragma unroll
+                    for (int c = 4; c < 64; c += 2) {
+                        acc[(c / 2) & 3] = max3f(acc[(c / 2) & 3], __uint_as_float(s[c]), __uint_as_float(s[c + 1]));
+                        acc[4 + ((c / 2) & 3)] =
+                            max3f(acc[4 + ((c / 2) & 3)], __uint_as_float(s[64 + c]), __uint_as_float(s[64 + c + 1]));
+                    }
+                    const float m0 = fmaxf(fmaxf(acc[0], acc[1]), fmaxf(acc[2], acc[3]));
+                    const float m1 = fmaxf(fmaxf(acc[4], acc[5]), fmaxf(acc[6], acc[7]));
+                    mt = fmaxf(member ? m0 : -INFINITY, mem1 ? m1 : -INFINITY);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < TC; ++c)
+                        if (c < 64 ? (member && c < nvalid) : (mem1 && c - 64 < nv1))
+                            mt = fmaxf(mt, __uint_as_float(s[c]));
+                }
+            } else {
             if (full) {   // 3-input max tree: short dependency chains
                 float acc[8];
 #pragma unroll
@@ -441,6 +499,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 for (int c = 0; c < BKV; ++c)
                     if (c < nvalid) mt = fmaxf(mt, __uint_as_float(s[c]));
             }
+            }
             const float mt2 = mt * kScaleLog2;
             const bool need = mt2 > m_ref + kRescale;
             const bool corr = need && m_ref != -INFINITY;
@@ -450,7 +509,41 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             // p in fp32, packed to fp16 pairs in place: pair i lands in s[i], after s[2i],
             // s[2i+1] were read
             float rs = 0.f;
-            if (full) {
+            if constexpr (KB == 2) {
+                if (full) {
+                    // every column, then the halves this row's query block did not keep are
+                    // dropped from the sum and from P (their p may be inf: never used)
+                    float2 r2[4];   // [0, 1]: first half, [2, 3]: second half
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) r2[i] = make_float2(0.f, 0.f);
+                    const float2 scale2 = make_float2(kScaleLog2, kScaleLog2);
+                    const float2 shift2 = make_float2(-m_ref, -m_ref);
+#pragma unroll
+                    for (int c = 0; c < TC; c += 2) {
+                        const int i = c / 2;
+                        const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
+                                                    scale2, shift2);
+                        const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                        r2[(c < 64 ? 0 : 2) + (i & 1)] = __fadd2_rn(r2[(c < 64 ? 0 : 2) + (i & 1)], pr);
+                        s[i] = pack_half2(pr.x, pr.y);
+                    }
+                    const float r0 = (r2[0].x + r2[0].y) + (r2[1].x + r2[1].y);
+                    const float r1 = (r2[2].x + r2[2].y) + (r2[3].x + r2[3].y);
+                    rs = (member ? r0 : 0.f) + (mem1 ? r1 : 0.f);
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) s[i] = (i < 32 ? member : mem1) ? s[i] : 0u;
+                } else {
+#pragma unroll
+                    for (int c = 0; c < TC; c += 2) {
+                        const bool v0 = c < 64 ? (member && c < nvalid) : (mem1 && c - 64 < nv1);
+                        const bool v1 = c + 1 < 64 ? (member && c + 1 < nvalid) : (mem1 && c + 1 - 64 < nv1);
+                        const float p0 = v0 ? ex2_approx(fmaf(__uint_as_float(s[c]), kScaleLog2, -m_ref)) : 0.f;
+                        const float p1 = v1 ? ex2_approx(fmaf(__uint_as_float(s[c + 1]), kScaleLog2, -m_ref)) : 0.f;
+                        rs += p0 + p1;
+                        s[c / 2] = pack_half2(p0, p1);
+                    }
+                }
+            } else if (full) {
                 // packed fp32 pair arithmetic: half the issue slots of scalar FMA / add
                 float2 r2[4];   // independent partial sums
 #pragma unroll
@@ -497,7 +590,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
             }
 #pragma unroll
-            for (int c = 0; c < BKV / 64; ++c)
+            for (int c = 0; c < TC / 64; ++c)
                 tmem_st32(lane_base + kColP + 32 * c, *reinterpret_cast<const uint32_t(*)[32]>(&s[32 * c]));
             tmem_wait_st();
             tc_fence_before();
