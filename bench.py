@@ -97,19 +97,30 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------- helpers
+def kernel_source_hash() -> str:
+    """sha256 of the attention kernel's sources with comments and whitespace removed, so that
+    the stored traffic record stays valid across comment edits and goes stale on any code
+    change."""
+    import hashlib
+    import re
+    text = "".join(open(os.path.join(ROOT, "view_transformers_b200", "csrc", f)).read()
+                   for f in ("attn_tc.cu", "sm100.cuh", "tc_layout.cuh"))
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return hashlib.sha256(re.sub(r"\s+", "", text).encode()).hexdigest()
+
+
 def measured_traffic(w, path):
     """DRAM bytes per launch of the fused kernel from the committed ncu record, scaled to this
-    workload by patch tokens x heads; None when the kernel source changed since the capture."""
-    import hashlib
+    workload by patch tokens x heads; None when the kernel code changed since the capture."""
     if path != "fused":
         return None
     try:
         rec = json.load(open(os.path.join(ROOT, "profiles", "fused_traffic.json")))
-        src = b"".join(open(os.path.join(ROOT, "view_transformers_b200", "csrc", f), "rb").read()
-                       for f in ("attn_tc.cu", "sm100.cuh", "tc_layout.cuh"))
+        src_hash = kernel_source_hash()
     except (OSError, ValueError):
         return None
-    if hashlib.sha256(src).hexdigest() != rec.get("source_sha256"):
+    if src_hash != rec.get("source_sha256"):
         return None
     return rec["dram_bytes_per_launch"] * (w.n_patch * w.heads) / (rec["patch_tokens"] * rec["heads"])
 

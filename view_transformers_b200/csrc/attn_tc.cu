@@ -10,8 +10,8 @@
 //                      one online softmax: steps 4, 5(ii) and the merge in one pass -> out
 //
 // Inputs come from the packed workspace (pack.cu): per head, 64-wide rows of 128 bytes,
-// so each query tile (128 rows) and each key tile (BKV rows) is one 2D TMA box with the
-// 128-byte swizzle that the MMA descriptors expect.
+// so a query tile (128 rows) is one 2D TMA box with the 128-byte swizzle that the MMA
+// descriptors expect, and a 128-key tile is one box of b = 128 rows or two of b = 64.
 //
 // One CTA per work item, two CTAs per SM (112 KB of shared memory and 256 TMEM columns
 // each, so the softmax of one CTA overlaps the tensor-core work of the other). 6 warps:
