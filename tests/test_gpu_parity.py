@@ -153,6 +153,9 @@ EDGE = [
     # an odd number of (query tile, head) items at b = 128 (the fused kernel pairs them), with
     # uneven kept counts between the rows of a pair
     configs.Workload("odd_items_b128", 3, 777, 5, 3, 64, 128, 0.5, 0.5, "bf16", "five_percent"),
+    # more than 32 heads: the attention kernels keep the plain head order (no work ranking)
+    configs.Workload("many_heads_b128", 1, 300, 5, 40, 64, 128, 0.5, 0.0, "bf16", "five_percent"),
+    configs.Workload("many_heads_b64", 1, 300, 5, 40, 64, 64, 0.5, 0.5, "bf16", "five_percent"),
 ]
 
 
