@@ -334,16 +334,6 @@ def merge(o_a, lse_a, o_b, lse_b):
     return wa * o_a + wb * o_b, L
 
 
-def dense_attention(Q, K, V, chunk: int = 512):
-    """Eq. (1) over all N tokens, every head: the all-ones-mask comparator."""
-    N, H, d = Q.shape
-    out = np.empty((N, H, d))
-    for h in range(H):
-        for c in range(0, N, chunk):
-            out[c:c + chunk, h], _ = attend(Q[c:c + chunk, h], K[:, h], V[:, h])
-    return out
-
-
 # ----------------------------------------------------------------------------- whole layer
 
 @dataclass

@@ -53,6 +53,15 @@ def test_k_helpers_match_oracle(lib):
             assert _lib.bsa_k_from_density(B, d) == oracle.k_from_density(B, d)
 
 
+def test_k_from_density_golden_cases(lib):
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "k_from_density_cases.txt")
+    for line in open(path):
+        if line.strip() and not line.startswith("#"):
+            B, d, k = line.split()
+            assert _lib.bsa_k_from_density(int(B), float(d)) == int(k), line
+
+
 @pytest.mark.parametrize("seed", range(10))
 def test_head_budgets_match_oracle(lib, seed):
     rng = np.random.default_rng(seed)

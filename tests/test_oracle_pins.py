@@ -122,6 +122,18 @@ def test_k_from_rho_matches_exact_rational_floor():
             assert oracle.k_from_rho(B, float(rho)) == math.floor(B * (1 - Fraction(rho)))
 
 
+def test_k_from_density_golden_cases_with_the_one_block_floor():
+    """Hand-derived budgets, including densities whose floor is 0 (clamped to one block)
+    and products that land on an integer only in exact arithmetic (10 x 0.7, 100 x 0.29)."""
+    lines = _lines("k_from_density_cases.txt")
+    assert any(int(l.split()[2]) == 1 and math.floor(int(l.split()[0]) * Fraction(l.split()[1])) == 0
+               for l in lines)                                    # the clamp is exercised
+    for line in lines:
+        B, d, k = line.split()
+        assert oracle.k_from_density(int(B), float(d)) == int(k), line
+        assert min(int(B), max(1, math.floor(int(B) * Fraction(d)))) == int(k), line
+
+
 def test_water_fill_golden_cases():
     for line in _lines("water_fill_cases.txt"):
         s, total, cap, want = [x.split() for x in line.split("|")]
