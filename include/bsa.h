@@ -28,8 +28,9 @@
  *     Device pointers must be 16-byte aligned.
  *   - Every device call is asynchronous and ordered on `stream` (NULL = legacy stream).
  *   - status_dev: optional device int32 (NULL allowed). Kernels write the first device-
- *     side error (BSA_ERR_TIMEOUT, BSA_ERR_DEVICE_BOUNDS) there and skip the faulty
- *     access instead of faulting; read it with bsa_check_status. Zero it before use.
+ *     side error (BSA_ERR_TIMEOUT, BSA_ERR_DEVICE_BOUNDS, BSA_ERR_RANGE) there and skip
+ *     the faulty access instead of faulting; read it with bsa_check_status. Zero it
+ *     before use.
  *   - Host-side validation happens before any launch; on error nothing is launched.
  *     A failed launch returns BSA_ERR_CUDA.
  */
@@ -57,7 +58,10 @@ typedef enum {
     BSA_ERR_UNSUPPORTED = 2,   /* valid arguments outside what the kernels implement */
     BSA_ERR_CUDA = 3,          /* a CUDA runtime or driver call failed */
     BSA_ERR_TIMEOUT = 4,       /* device: a bounded wait ran out */
-    BSA_ERR_DEVICE_BOUNDS = 5  /* device: an out-of-range index was rejected */
+    BSA_ERR_DEVICE_BOUNDS = 5, /* device: an out-of-range index was rejected */
+    BSA_ERR_RANGE = 6          /* device: an input value outside the range the kernels take
+                                  (a bf16 V element of magnitude >= 65536, inf or NaN: the
+                                  fp16 operand of the P.V product cannot hold it) */
 } bsa_status;
 
 typedef enum { BSA_F32 = 0, BSA_BF16 = 1 } bsa_dtype;
@@ -120,6 +124,9 @@ BSA_API bsa_status bsa_predict_mask(const bsa_layout* layout, const float* pq, c
  * multiple of 128 and special rows padded likewise, padding zeroed; Q and K stay bf16,
  * V is converted to fp16 (the operand type of the P.V product; exact for |v| in
  * [2^-14, 65504], smaller magnitudes lose precision, larger ones overflow).
+ * A V element of magnitude >= 65536 (or inf / NaN), which fp16 cannot hold, is reported
+ * as BSA_ERR_RANGE through status_dev (the layer's output is then not valid); magnitudes
+ * below 2^-14 become fp16 subnormals, with an absolute error below 2^-25.
  * Must run after Q, K, V hold the layer's values and before bsa_block_sparse_attn /
  * bsa_special_dense on the same stream. Not needed (no-op) for f32 layouts.
  *   q, k, v          : device, [N, H, d] bf16
@@ -133,7 +140,7 @@ BSA_API bsa_status bsa_pack_qkv(const bsa_layout* layout, const void* q, const v
  * Packing and step 1 in one pass: the packed workspace of bsa_pack_qkv and the pooled
  * pq, pk of bsa_pool_qk (same layouts and values up to fp32 summation order), reading
  * Q and K from HBM once for both. For f32 layouts only the pooling runs (workspace
- * ignored, may be NULL).
+ * ignored, may be NULL). V values outside the fp16 range are reported as in bsa_pack_qkv.
  *   q, k, v          : device, [N, H, d] of layout->dtype
  *   workspace        : bf16: device, at least bsa_workspace_size() bytes, 1024-byte aligned
  *   pq, pk           : device, float32 [H, B, d] and [H, d, B]
@@ -221,6 +228,7 @@ BSA_API bsa_status bsa_block_sparse_attn_fused(const bsa_layout* layout, const v
  * the kept blocks), but keeps the packed copy and the partial results in one static
  * device array of BSA_NOALLOC_SCRATCH_BYTES inside the library instead of a workspace.
  * The array exists on every GPU that loads the library until the process exits.
+ *   - V values outside the fp16 range are reported through status_dev as in bsa_pack_qkv.
  *   - Layers whose packed data (bsa_workspace_size) exceed BSA_NOALLOC_SCRATCH_BYTES are
  *     rejected with BSA_ERR_UNSUPPORTED before anything is launched.
  *   - No memory is allocated or freed. The first call on a device looks up the device

@@ -25,9 +25,14 @@ def oracle_layout(w: configs.Workload) -> oracle.Layout:
 
 
 def head_density(w: configs.Workload, x: synth.LayerInputs):
+    """Per-head densities from the library's own capped water-filling (the step the
+    product runs), checked against the oracle's on the way."""
     if x.scores is None:
         return None
-    return oracle.water_fill(x.scores, w.heads * (1.0 - w.rho), 1.0)
+    from view_transformers_b200 import _lib
+    dens = _lib.bsa_head_budgets(x.scores, w.rho, 1.0)
+    assert np.allclose(dens, oracle.water_fill(x.scores, w.heads * (1.0 - w.rho), 1.0), rtol=0, atol=1e-12)
+    return dens
 
 
 def run_gpu(w: configs.Workload, x: synth.LayerInputs, density=None, tamper=None):

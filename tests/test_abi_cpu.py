@@ -32,7 +32,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    for code in range(6):
+    for code in range(7):
         assert _lib.status_string(code)
     assert _lib.status_string(99) == "unknown status"
 

@@ -14,7 +14,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libbsa.so")
 HEADER = os.path.join(os.path.dirname(PKG), "include", "bsa.h")
 
-BSA_OK, BSA_ERR_INVALID_ARG, BSA_ERR_UNSUPPORTED, BSA_ERR_CUDA, BSA_ERR_TIMEOUT, BSA_ERR_DEVICE_BOUNDS = range(6)
+(BSA_OK, BSA_ERR_INVALID_ARG, BSA_ERR_UNSUPPORTED, BSA_ERR_CUDA, BSA_ERR_TIMEOUT, BSA_ERR_DEVICE_BOUNDS,
+ BSA_ERR_RANGE) = range(7)
 BSA_F32, BSA_BF16 = 0, 1
 DTYPES = {"f32": BSA_F32, "bf16": BSA_BF16}
 

@@ -27,9 +27,9 @@ cudaError_t launch_attn_tc(const Geo& g, int mode, const void* ws, const uint16_
                            const int32_t* kv_cnt, float* o_part, float* lse_part, void* out,
                            int32_t* status, cudaStream_t st);
 cudaError_t launch_pack_pool(const Geo& g, const void* q, const void* k, const void* v, void* ws,
-                             float* pq, float* pk, cudaStream_t st);
+                             float* pq, float* pk, int32_t* status, cudaStream_t st);
 cudaError_t launch_pack(const Geo& g, const void* q, const void* k, const void* v, void* ws,
-                        cudaStream_t st);
+                        int32_t* status, cudaStream_t st);
 
 namespace {
 
@@ -102,6 +102,7 @@ const char* bsa_status_string(bsa_status s) {
         case BSA_ERR_CUDA: return "CUDA error";
         case BSA_ERR_TIMEOUT: return "device wait timed out";
         case BSA_ERR_DEVICE_BOUNDS: return "device index out of range";
+        case BSA_ERR_RANGE: return "input value outside the range of the kernels' operand type";
     }
     return "unknown status";
 }
@@ -127,7 +128,6 @@ bsa_status bsa_workspace_size(const bsa_layout* layout, size_t* bytes) {
 bsa_status bsa_pack_qkv(const bsa_layout* layout, const void* q, const void* k, const void* v,
                         void* workspace, size_t workspace_bytes, int32_t* status_dev,
                         bsa_stream_t stream) {
-    (void)status_dev;
     Geo g;
     bsa_status s = make_geo(layout, &g);
     if (s != BSA_OK) return s;
@@ -135,13 +135,12 @@ bsa_status bsa_pack_qkv(const bsa_layout* layout, const void* q, const void* k, 
     if (!q || !k || !v || !aligned16(q) || !aligned16(k) || !aligned16(v)) return BSA_ERR_INVALID_ARG;
     s = check_ws(g, workspace, workspace_bytes);
     if (s != BSA_OK) return s;
-    return from_cuda(launch_pack(g, q, k, v, workspace, reinterpret_cast<cudaStream_t>(stream)));
+    return from_cuda(launch_pack(g, q, k, v, workspace, status_dev, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 bsa_status bsa_pack_pool_qkv(const bsa_layout* layout, const void* q, const void* k, const void* v,
                              void* workspace, size_t workspace_bytes, float* pq, float* pk,
                              int32_t* status_dev, bsa_stream_t stream) {
-    (void)status_dev;
     Geo g;
     bsa_status s = make_geo(layout, &g);
     if (s != BSA_OK) return s;
@@ -153,11 +152,11 @@ bsa_status bsa_pack_pool_qkv(const bsa_layout* layout, const void* q, const void
     s = check_ws(g, workspace, workspace_bytes);
     if (s != BSA_OK) return s;
     if (!tc_supported(g)) {   // the one-pass kernel needs whole blocks per 128-row tile
-        cudaError_t e = launch_pack(g, q, k, v, workspace, st);
+        cudaError_t e = launch_pack(g, q, k, v, workspace, status_dev, st);
         if (e == cudaSuccess) e = launch_pool(g, layout->dtype, q, k, pq, pk, st);
         return from_cuda(e);
     }
-    return from_cuda(launch_pack_pool(g, q, k, v, workspace, pq, pk, st));
+    return from_cuda(launch_pack_pool(g, q, k, v, workspace, pq, pk, status_dev, st));
 }
 
 bsa_status bsa_k_from_rho(int32_t num_blocks, double rho, int32_t* k) {
@@ -223,7 +222,7 @@ bsa_status bsa_check_status(int32_t* status_dev, bsa_stream_t stream) {
     if (cudaStreamSynchronize(st) != cudaSuccess) return BSA_ERR_CUDA;
     if (v != 0 && cudaMemsetAsync(status_dev, 0, sizeof(int32_t), st) != cudaSuccess) return BSA_ERR_CUDA;
     if (v == 0) return BSA_OK;
-    if (v == BSA_ERR_TIMEOUT || v == BSA_ERR_DEVICE_BOUNDS) return (bsa_status)v;
+    if (v == BSA_ERR_TIMEOUT || v == BSA_ERR_DEVICE_BOUNDS || v == BSA_ERR_RANGE) return (bsa_status)v;
     return BSA_ERR_CUDA;
 }
 

@@ -15,7 +15,7 @@ cudaError_t launch_attn_tc(const Geo& g, int mode, const void* ws, const uint16_
                            const int32_t* kv_cnt, float* o_part, float* lse_part, void* out,
                            int32_t* status, cudaStream_t st);
 cudaError_t launch_pack(const Geo& g, const void* q, const void* k, const void* v, void* ws,
-                        cudaStream_t st);
+                        int32_t* status, cudaStream_t st);
 bsa_status make_geo_checked(const bsa_layout* L, Geo* g);
 }  // namespace bsa
 
@@ -66,7 +66,7 @@ extern "C" bsa_status bsa_attention_noalloc(const bsa_layout* layout, const void
     if (scratch_address(&base) != cudaSuccess) return BSA_ERR_CUDA;
     void* ws = reinterpret_cast<void*>((reinterpret_cast<uintptr_t>(base) + 1023) & ~uintptr_t(1023));
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (launch_pack(g, q, k, v, ws, st) != cudaSuccess) return BSA_ERR_CUDA;
+    if (launch_pack(g, q, k, v, ws, status_dev, st) != cudaSuccess) return BSA_ERR_CUDA;
     if (g.Ns > 0 &&
         launch_attn_tc(g, 2, ws, nullptr, nullptr, nullptr, nullptr, out, status_dev, st) != cudaSuccess)
         return BSA_ERR_CUDA;

@@ -7,7 +7,8 @@
 // query tile (128 rows) and key tile (b rows) is one contiguous 2D TMA box, so no tile
 // straddles a frame boundary, and V is already in the operand type of the P.V product
 // (P is rounded to fp16, whose 11-bit significand keeps the output error well inside
-// the bf16 tolerance; bf16 -> fp16 is exact for |v| in [2^-14, 65504]).
+// the bf16 tolerance; bf16 -> fp16 is exact for |v| in [2^-14, 65504]). A V element that
+// fp16 cannot hold (|v| >= 65536, inf, NaN) is reported as BSA_ERR_RANGE in the status word.
 //
 // HBM-bound: Q, K, V read once, written once (plus zero padding).
 #include "common.cuh"
@@ -16,10 +17,21 @@
 namespace bsa {
 namespace {
 
+// True when a bf16 pair holds an element fp16 cannot hold: magnitude >= 2^16 (bf16 has no
+// value between 65280 and 65536, and fp16's largest finite value is 65504), inf or NaN.
+__device__ __forceinline__ bool beyond_f16(uint32_t pair) {
+    return (pair & 0x7fffu) >= 0x4780u || ((pair >> 16) & 0x7fffu) >= 0x4780u;
+}
+
+__device__ __forceinline__ bool beyond_f16(uint4 w) {
+    return beyond_f16(w.x) || beyond_f16(w.y) || beyond_f16(w.z) || beyond_f16(w.w);
+}
+
 __global__ void __launch_bounds__(256)
 pack_kernel(Geo g, PackedLayout pl, const __nv_bfloat16* __restrict__ q,
             const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
-            unsigned char* __restrict__ ws) {
+            unsigned char* __restrict__ ws, int32_t* status) {
+    bool out_of_range = false;
     const int chunks = g.H * 8;                      // 16-byte chunks per token row
     const size_t rows = (size_t)pl.np_pad + pl.ns_pad;
     const size_t total = rows * chunks;
@@ -49,6 +61,7 @@ pack_kernel(Geo g, PackedLayout pl, const __nv_bfloat16* __restrict__ q,
             vq = __ldg(reinterpret_cast<const uint4*>(q + off));
             vk = __ldg(reinterpret_cast<const uint4*>(k + off));
             const uint4 w = __ldg(reinterpret_cast<const uint4*>(v + off));
+            out_of_range |= beyond_f16(w);
             const uint32_t in[4] = {w.x, w.y, w.z, w.w};
             uint32_t o[4];
 #pragma unroll
@@ -64,6 +77,7 @@ pack_kernel(Geo g, PackedLayout pl, const __nv_bfloat16* __restrict__ q,
         *reinterpret_cast<uint4*>(ws + base_k + dst) = vk;
         *reinterpret_cast<uint4*>(ws + base_v + dst) = vv;
     }
+    if (out_of_range) record_error(status, BSA_ERR_RANGE);
 }
 
 // Packing with block pooling folded in: the same copies as pack_kernel, plus the block
@@ -104,8 +118,10 @@ __device__ __forceinline__ void add_bf16x8(float* acc, uint4 w) {
 __global__ void __launch_bounds__(256)
 pack_pool_kernel(Geo g, PackedLayout pl, const __nv_bfloat16* __restrict__ q,
                  const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
-                 unsigned char* __restrict__ ws, float* __restrict__ pq, float* __restrict__ pk) {
+                 unsigned char* __restrict__ ws, float* __restrict__ pq, float* __restrict__ pk,
+                 int32_t* status) {
     __shared__ float red[2][kPhases][kPoolHeads * 64];   // per-phase sums of Q and K
+    bool out_of_range = false;
     const int groups = (g.H + kPoolHeads - 1) / kPoolHeads;
     const int p_tiles = pl.np_pad / 128;
     const int units = (p_tiles + pl.ns_pad / 128) * groups;
@@ -136,7 +152,9 @@ pack_pool_kernel(Geo g, PackedLayout pl, const __nv_bfloat16* __restrict__ q,
                     const size_t off = (size_t)src_row * g.H * 64 + (size_t)h * 64 + c8 * 8;
                     vq = __ldg(reinterpret_cast<const uint4*>(q + off));
                     vk = __ldg(reinterpret_cast<const uint4*>(k + off));
-                    vv = bf16x8_to_f16x8(__ldg(reinterpret_cast<const uint4*>(v + off)));
+                    const uint4 w = __ldg(reinterpret_cast<const uint4*>(v + off));
+                    out_of_range |= beyond_f16(w);
+                    vv = bf16x8_to_f16x8(w);
                     if (patch) { add_bf16x8(sq, vq); add_bf16x8(sk, vk); }
                 }
                 const size_t dst = (dst_base + r) * 128 + c8 * 16;
@@ -176,27 +194,28 @@ pack_pool_kernel(Geo g, PackedLayout pl, const __nv_bfloat16* __restrict__ q,
             __syncthreads();
         }
     }
+    if (out_of_range) record_error(status, BSA_ERR_RANGE);
 }
 }  // namespace
 
 cudaError_t launch_pack(const Geo& g, const void* q, const void* k, const void* v, void* ws,
-                        cudaStream_t st) {
+                        int32_t* status, cudaStream_t st) {
     const PackedLayout pl = packed_layout(g);
     pack_kernel<<<num_sms() * 8, 256, 0, st>>>(g, pl, static_cast<const __nv_bfloat16*>(q),
                                                static_cast<const __nv_bfloat16*>(k),
                                                static_cast<const __nv_bfloat16*>(v),
-                                               static_cast<unsigned char*>(ws));
+                                               static_cast<unsigned char*>(ws), status);
     return cudaGetLastError();
 }
 
 cudaError_t launch_pack_pool(const Geo& g, const void* q, const void* k, const void* v, void* ws,
-                             float* pq, float* pk, cudaStream_t st) {
+                             float* pq, float* pk, int32_t* status, cudaStream_t st) {
     const PackedLayout pl = packed_layout(g);
     const int groups = (g.H + kPoolHeads - 1) / kPoolHeads;
     const int units = (pl.np_pad / 128 + pl.ns_pad / 128) * groups;
     pack_pool_kernel<<<units, 256, 0, st>>>(
         g, pl, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-        static_cast<const __nv_bfloat16*>(v), static_cast<unsigned char*>(ws), pq, pk);
+        static_cast<const __nv_bfloat16*>(v), static_cast<unsigned char*>(ws), pq, pk, status);
     return cudaGetLastError();
 }
 
