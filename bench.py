@@ -174,10 +174,10 @@ def step_calls(L, q, k, v, path: str):
     status = b.status.data_ptr()
     lay = L.layout
     qp, kp, vp = q.data_ptr(), k.data_ptr(), v.data_ptr()
-    mask = ("mask", lambda: _lib.bsa_predict_mask(lay, b.pq.data_ptr(), b.pk.data_ptr(), L.rho, L.tau,
-                                                  L.head_density, b.mask_bits.data_ptr(), b.kv_idx.data_ptr(),
-                                                  b.kv_cnt.data_ptr(), status, sp), 1)
-    if path == "fused":
+    mask = ("mask", lambda: L._select(sp), 1)
+    if path == "fused" and L.selector in ("random", "uniform"):   # no pooled means needed
+        calls = [("pack", lambda: _lib.bsa_pack_qkv(lay, qp, kp, vp, L.ws_ptr, L.ws_bytes, status, sp), 1), mask]
+    elif path == "fused":
         calls = [
             ("pack_pool", lambda: _lib.bsa_pack_pool_qkv(lay, qp, kp, vp, L.ws_ptr, L.ws_bytes, b.pq.data_ptr(),
                                                          b.pk.data_ptr(), status, sp), 1),
@@ -270,13 +270,20 @@ def oracle_layer_sample(w, x, budget_s: float, seed: int = 7):
 
 
 def _oracle_layer_sample(oracle, w, x, budget_s, seed):
-    lay = oracle.Layout(w.frames, w.tokens_per_frame, w.special_per_frame, w.heads, w.head_dim, w.block)
+    from oracle import selectors
+    lay = oracle.Layout(w.frames, w.tokens_per_frame, w.layer_special, w.heads, w.head_dim, w.block)
     t0 = time.perf_counter()
     Q, K = oracle.to_f64(x.q, w.dtype), oracle.to_f64(x.k, w.dtype)
-    PQ, PK = oracle.pool(Q, lay), oracle.pool(K, lay)
     dens = None if x.scores is None else oracle.water_fill(x.scores, w.heads * (1 - w.rho), 1.0)
     kh = oracle.head_k(lay, w.rho, dens)
-    m = oracle.predict_mask(PQ, PK, lay.head_dim, kh, w.tau)
+    if w.selector == "predict":
+        selected = oracle.predict_mask(oracle.pool(Q, lay), oracle.pool(K, lay), lay.head_dim, kh, w.tau).selected
+    elif w.selector == "random":
+        selected = selectors.random_mask(lay, kh, w.seed)
+    elif w.selector == "uniform":
+        selected = selectors.uniform_mask(lay, w.stride)
+    else:
+        selected = selectors.probe_mask(Q, K, lay, kh)[1]
     t_mask = time.perf_counter() - t0
     V = oracle.to_f64(x.v, w.dtype)
     g = np.random.default_rng(seed)
@@ -286,7 +293,7 @@ def _oracle_layer_sample(oracle, w, x, budget_s, seed):
     sr = oracle.special_rows(lay)
     for h, i in pairs:
         rows = oracle.patch_rows(lay)[slice(*oracle.block_bounds(lay, i))]
-        keys = np.concatenate([sr, oracle.patch_keys_of(lay, m.selected[h, i])])
+        keys = np.concatenate([sr, oracle.patch_keys_of(lay, selected[h, i])])
         oracle.attend(Q[rows, h], K[keys, h], V[keys, h])
         done += 1
         if time.perf_counter() - t1 > budget_s * 0.8:
@@ -326,11 +333,22 @@ def reference_arm(args, w):
     print(json.dumps(line), flush=True)
 
 
+SELECTOR_TEXT = {
+    "predict": "",
+    "random": ", random blocks (k_h per row, Philox4x32-10 keys, seed {seed})",
+    "uniform": ", fixed-stride uniform sampling (every {stride}th block)",
+    "probe": ", query-probe Top-K (mean-query scores, k_h per head)",
+}
+
+
 def workload_config(w):
     return {"workload": f"{w.name}: {w.frames} frames x ({w.patch_per_frame} patch + {w.special_per_frame} special)"
                         f" tokens, {w.heads} heads, d={w.head_dim}, b={w.block}, rho={w.rho}, tau={w.tau}"
                         + (", per-head budgets (LogNormal(0,1) scores, capped water-filling, cap 1)"
-                           if w.head_budgets else ""),
+                           if w.head_budgets else "")
+                        + SELECTOR_TEXT[w.selector].format(seed=w.seed, stride=w.stride)
+                        + (", special tokens read as patch tokens (no dense special path)"
+                           if w.sparse_specials else ""),
             "frames": w.frames, "tokens_per_frame": w.tokens_per_frame, "heads": w.heads, "head_dim": w.head_dim,
             "block": w.block, "rho": w.rho, "tau": w.tau, "global_batch": 1, "seq_len": w.n_tokens,
             "parallelism": "replicas",
@@ -476,15 +494,16 @@ def main():
 
     kv_cnt = L.buf.kv_cnt.cpu().numpy()
     kv_idx = L.buf.kv_idx.cpu().numpy().view(np.uint16)
-    f_sparse = sparse_flops(kv_cnt, kv_idx, w)
-    f_special = special_flops(w)
-    density_real = f_sparse / (4 * w.head_dim * w.heads * float(w.n_patch) ** 2)
+    wl = w.layer_view()     # token split as the layer reads it
+    f_sparse = sparse_flops(kv_cnt, kv_idx, wl)
+    f_special = special_flops(wl)
+    density_real = f_sparse / (4 * wl.head_dim * wl.heads * float(wl.n_patch) ** 2)
     stage_ms = {k_: float(np.mean(vs)) for k_, vs in per_stage.items()}
 
     # dense comparator: the same kernels with every block kept
     dense_ms, dense_stage = None, {}
     if args.dense_steps > 0:
-        Ld = layer.BlockSparseLayer.for_workload(w.with_(rho=0.0, tau=0.0, head_budgets=False))
+        Ld = layer.BlockSparseLayer.for_workload(w.with_(rho=0.0, tau=0.0, head_budgets=False, selector="predict"))
         run_forward(torch, Ld, q, k, v, 2, path)
         dense_ms = run_forward(torch, Ld, q, k, v, args.dense_steps, path) / args.dense_steps
         dense_stage, _, _ = run_steps(torch, Ld, q, k, v, args.dense_steps, path)
@@ -506,9 +525,9 @@ def main():
     sparse_ms = float(np.mean(fused_kernel_ms)) if fused_kernel_ms else stage_ms["sparse"]
     # algorithmic work of the timed sparse kernel: kept patch-patch entries, plus the
     # patch-to-special entries when the special keys are fused into it
-    f_kernel = f_sparse + (4.0 * w.head_dim * w.heads * w.n_patch * w.n_special if path == "fused" else 0.0)
+    f_kernel = f_sparse + (4.0 * wl.head_dim * wl.heads * wl.n_patch * wl.n_special if path == "fused" else 0.0)
     achieved = f_kernel / (sparse_ms * 1e-3) / 1e12
-    sb = stage_bytes(w)
+    sb = stage_bytes(wl)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": False, "scaling": "weak",

@@ -118,6 +118,41 @@ BSA_API bsa_status bsa_predict_mask(const bsa_layout* layout, const float* pq, c
                             int32_t* status_dev, bsa_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
+ * Alternative block selectors. Each writes the same outputs as bsa_predict_mask (mask_bits
+ * optional, kv_idx ascending in the first kv_cnt entries of each row, kv_cnt), so that the
+ * same attention entry points compute the layer under them. k_h is computed as in
+ * bsa_predict_mask from rho and the optional host head_density (validated the same way).
+ *
+ * Random selection -- the "Random" rows of the ablation in "Block-Sparse Global Attention
+ * for Efficient Multi-View Geometry Transformers", 消融实验 (图 10): every row (h, i) keeps
+ * k_h blocks drawn uniformly without replacement. Block j of row (h, i) gets the 32-bit key
+ * word 0 of Philox4x32-10 (Salmon et al., "Parallel Random Numbers: As Easy as 1, 2, 3",
+ * SC 2011) at counter (j, i, h, 0) under key (seed mod 2^32, seed >> 32); the row keeps the
+ * k_h blocks of smallest (key, j). Deterministic in (layout, k_h, seed).
+ */
+BSA_API bsa_status bsa_random_mask(const bsa_layout* layout, double rho, const double* head_density,
+                                   uint64_t seed, uint32_t* mask_bits, uint16_t* kv_idx, int32_t* kv_cnt,
+                                   int32_t* status_dev, bsa_stream_t stream);
+
+/* Fixed-stride uniform sampling -- "SAF3R: Dynamic Sparse Attention for Feed-Forward 3D
+ * Reconstruction Transformers", 四、1. 均匀采样核 (scanning heads): every row keeps the patch
+ * key blocks j = 0, stride, 2 stride, ... (ceil(B / stride) blocks).
+ *   stride : >= 1 */
+BSA_API bsa_status bsa_uniform_mask(const bsa_layout* layout, int32_t stride, uint32_t* mask_bits,
+                                    uint16_t* kv_idx, int32_t* kv_cnt, int32_t* status_dev,
+                                    bsa_stream_t stream);
+
+/* Query-probe Top-K -- the same page, 四、1. Query-Probe Top-K 核 and its acceleration in 四、3.:
+ * q_bar_h = the mean of the patch queries of head h (taken from the pooled means weighted by
+ * the block sizes, in fp64); block j's probe score is q_bar_h . pk[h, :, j] / sqrt(d) (the
+ * column means of Q K^T / sqrt(d) averaged over the block's keys), rounded to fp32; the k_h
+ * blocks of highest score (ties to the lower index) are kept by every query block of head h.
+ *   pq, pk : device, float32 [H, B, d] and [H, d, B] (from bsa_pool_qk / bsa_pack_pool_qkv) */
+BSA_API bsa_status bsa_probe_mask(const bsa_layout* layout, const float* pq, const float* pk, double rho,
+                                  const double* head_density, uint32_t* mask_bits, uint16_t* kv_idx,
+                                  int32_t* kv_cnt, int32_t* status_dev, bsa_stream_t stream);
+
+/* ---------------------------------------------------------------------------------
  * Packing (prepares steps 4 and 5 for bf16 layers; the token split of 关键设计 3 made
  * physical). Copies the patch tokens and the special tokens of Q, K and V into a
  * head-major workspace: per head, rows of d = 64 elements, patch rows padded to a

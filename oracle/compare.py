@@ -86,3 +86,36 @@ def nmse_per_head(x: np.ndarray, ref: np.ndarray) -> np.ndarray:
     num = ((x - ref) ** 2).sum(axis=(0, 2))
     den = (ref ** 2).sum(axis=(0, 2))
     return num / np.maximum(den, 1e-300)
+
+
+def compare_probe(scores: np.ndarray, scale: np.ndarray, k_per_head, device_selected: np.ndarray,
+                  rel: float = 2e-5) -> MaskReport:
+    """Query-probe Top-K rule ("SAF3R: Dynamic Sparse Attention for Feed-Forward 3D
+    Reconstruction Transformers", 四、1. and 四、3.): per head, the device keeps k_h blocks, and
+    every block where it differs from the oracle's fp64 top-k has an oracle score within
+    rel * (scale_j + scale_cut) of the oracle's k-th score, where scale_j bounds the size of
+    the terms of block j's score (sum_d |q_bar_d| |P_b(K)_jd| / sqrt(d)).
+    scores, scale: [H, B]; device_selected: [H, B] bool (one row per head)."""
+    rep = MaskReport()
+    H, B = scores.shape
+    rep.rows = H
+    for h in range(H):
+        k = min(int(k_per_head[h]), B)
+        order = np.argsort(-scores[h], kind="stable")
+        ref = np.zeros(B, dtype=bool)
+        ref[order[:k]] = True
+        dev = device_selected[h]
+        if np.array_equal(ref, dev):
+            rep.exact += 1
+            continue
+        ok = int(dev.sum()) == k and k > 0
+        if ok:
+            cut = order[k - 1]
+            diff = np.nonzero(ref ^ dev)[0]
+            ok = bool(np.all(np.abs(scores[h, diff] - scores[h, cut]) <= rel * (scale[h, diff] + scale[h, cut])))
+        if ok:
+            rep.exempt += 1
+        else:
+            rep.failed += 1
+            rep.failures.append((h, k, int(dev.sum())))
+    return rep

@@ -118,6 +118,14 @@ def probe_block_scores(Q: np.ndarray, K: np.ndarray, lay: Layout) -> np.ndarray:
     return out
 
 
+def probe_score_scale(Q: np.ndarray, K: np.ndarray, lay: Layout) -> np.ndarray:
+    """[H, B]: sum_d |q_bar_d| |P_b(K)_jd| / sqrt(d), the size of the terms of each block's
+    probe score (the conditioning of its floating-point evaluation)."""
+    from .bsa_oracle import pool
+    qbar = mean_query(Q, lay)
+    return np.einsum("hd,hjd->hj", np.abs(qbar), np.abs(pool(K.astype(np.float64), lay))) / math.sqrt(lay.head_dim)
+
+
 def probe_mask(Q: np.ndarray, K: np.ndarray, lay: Layout, k_per_head):
     """Query-probe Top-K [SAF3R 四、1., 四、3.]: per head, the k_h blocks of highest probe score
     (ties to the lower index), kept by every query block. Returns (scores [H, B], mask)."""

@@ -44,6 +44,9 @@ _SIGS = {
     "bsa_merge": [_LP, _vp, _vp, _vp, _vp, _vp, _i32p, _st],
     "bsa_block_sparse_attn_fused": [_LP, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp, _i32p, _st],
     "bsa_attention_noalloc": [_LP, _vp, _vp, _vp, _vp, _vp, _vp, _i32p, _st],
+    "bsa_random_mask": [_LP, ctypes.c_double, ctypes.c_void_p, ctypes.c_uint64, _vp, _vp, _vp, _i32p, _st],
+    "bsa_uniform_mask": [_LP, ctypes.c_int32, _vp, _vp, _vp, _i32p, _st],
+    "bsa_probe_mask": [_LP, _vp, _vp, ctypes.c_double, ctypes.c_void_p, _vp, _vp, _vp, _i32p, _st],
     "bsa_num_blocks": [_LP, ctypes.POINTER(ctypes.c_int32)],
     "bsa_workspace_size": [_LP, ctypes.POINTER(ctypes.c_size_t)],
     "bsa_k_from_rho": [ctypes.c_int32, ctypes.c_double, ctypes.POINTER(ctypes.c_int32)],
@@ -155,6 +158,30 @@ def bsa_predict_mask(layout, pq, pk, rho, tau, head_density, mask_bits, kv_idx, 
     _check("bsa_predict_mask", load().bsa_predict_mask(ctypes.byref(layout), pq, pk, rho, tau,
                                                        ctypes.cast(dens, ctypes.c_void_p) if dens else None,
                                                        mask_bits, kv_idx, kv_cnt, status, stream))
+
+
+def _densities(head_density):
+    if head_density is None:
+        return None, None
+    dens = (ctypes.c_double * len(head_density))(*[float(x) for x in head_density])
+    return dens, ctypes.cast(dens, ctypes.c_void_p)
+
+
+def bsa_random_mask(layout, rho, head_density, seed, mask_bits, kv_idx, kv_cnt, status=0, stream=0) -> None:
+    keep, dens = _densities(head_density)
+    _check("bsa_random_mask", load().bsa_random_mask(ctypes.byref(layout), rho, dens, int(seed), mask_bits,
+                                                     kv_idx, kv_cnt, status, stream))
+
+
+def bsa_uniform_mask(layout, stride, mask_bits, kv_idx, kv_cnt, status=0, stream=0) -> None:
+    _check("bsa_uniform_mask", load().bsa_uniform_mask(ctypes.byref(layout), int(stride), mask_bits, kv_idx,
+                                                       kv_cnt, status, stream))
+
+
+def bsa_probe_mask(layout, pq, pk, rho, head_density, mask_bits, kv_idx, kv_cnt, status=0, stream=0) -> None:
+    keep, dens = _densities(head_density)
+    _check("bsa_probe_mask", load().bsa_probe_mask(ctypes.byref(layout), pq, pk, rho, dens, mask_bits, kv_idx,
+                                                   kv_cnt, status, stream))
 
 
 def bsa_pack_qkv(layout, q, k, v, workspace, workspace_bytes, status=0, stream=0) -> None:

@@ -30,6 +30,25 @@ class Workload:
     planting: str          # "tiny" (permuted cross-frame copies) or "five_percent"
     head_budgets: bool = False  # per-head densities from capped water-filling
     seed: int = 0
+    # block selector: "predict" (pooled softmax + dual threshold), "random" (k_h uniformly
+    # random blocks), "uniform" (every `stride`-th block), "probe" (mean-query Top-K)
+    selector: str = "predict"
+    stride: int = 4
+    # the ablation without the dense special path: the layer reads the S special tokens of
+    # every frame as patch tokens (pooled and sparsified with them)
+    sparse_specials: bool = False
+
+    @property
+    def layer_special(self) -> int:
+        """Special tokens per frame as the layer reads them."""
+        return 0 if self.sparse_specials else self.special_per_frame
+
+    def layer_view(self) -> "Workload":
+        """The workload as the layer reads it (the inputs are drawn from `self`): with
+        sparse_specials every token of a frame is a patch token."""
+        if not self.sparse_specials:
+            return self
+        return replace(self, patch_per_frame=self.tokens_per_frame, special_per_frame=0, sparse_specials=False)
 
     @property
     def tokens_per_frame(self) -> int:
@@ -72,5 +91,20 @@ LONG500 = Workload("long500", 500, 777, 5, 16, 64, 128, 0.9, 0.95, "bf16", "five
 TINY_TAU0 = TINY.with_(name="tiny_tau0", tau=0.0)
 SWEEP_TAU0 = SWEEP_R75.with_(name="sweep_tau0", tau=0.0)
 
+# Ablation rows of "Block-Sparse Global Attention for Efficient Multi-View Geometry
+# Transformers", 消融实验 (图 10), at the 100-frame shape: CDF threshold alone (no Top-K
+# floor: rho = 1, k = 0; tau = 0.25 keeps about a quarter of the blocks on these inputs),
+# without the dense special path, and random selection with and without it (same k_h).
+CDF_ONLY100 = PERHEAD100.with_(name="cdf_only100", head_budgets=False, rho=1.0, tau=0.25)
+NOSPECIAL100 = PERHEAD100.with_(name="nospecial100", sparse_specials=True)
+RANDOM100 = PERHEAD100.with_(name="random100", selector="random")
+RANDOM_NOSPECIAL100 = PERHEAD100.with_(name="random_nospecial100", selector="random", sparse_specials=True)
+# Key selectors of "SAF3R: Dynamic Sparse Attention for Feed-Forward 3D Reconstruction
+# Transformers", 四、1.: fixed-stride uniform sampling (every 4th block: 25% kept) and the
+# query-probe Top-K (the per-head budgets of the 100-frame workload).
+UNIFORM100 = PERHEAD100.with_(name="uniform100", selector="uniform", stride=4, head_budgets=False)
+PROBE100 = PERHEAD100.with_(name="probe100", selector="probe")
+
 ALL = {w.name: w for w in (TINY, VGGT518, SWEEP_R50, SWEEP_R75, SWEEP_R90, PERHEAD100,
-                           PERHEAD100_TAU95, LONG500, TINY_TAU0, SWEEP_TAU0)}
+                           PERHEAD100_TAU95, LONG500, TINY_TAU0, SWEEP_TAU0, CDF_ONLY100, NOSPECIAL100,
+                           RANDOM100, RANDOM_NOSPECIAL100, UNIFORM100, PROBE100)}

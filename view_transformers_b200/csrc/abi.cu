@@ -30,6 +30,12 @@ cudaError_t launch_pack_pool(const Geo& g, const void* q, const void* k, const v
                              float* pq, float* pk, int32_t* status, cudaStream_t st);
 cudaError_t launch_pack(const Geo& g, const void* q, const void* k, const void* v, void* ws,
                         int32_t* status, cudaStream_t st);
+cudaError_t launch_random_mask(const Geo& g, const int* k_per_head, uint64_t seed, uint32_t* mask_bits,
+                               uint16_t* kv_idx, int32_t* kv_cnt, cudaStream_t st);
+cudaError_t launch_uniform_mask(const Geo& g, int stride, uint32_t* mask_bits, uint16_t* kv_idx, int32_t* kv_cnt,
+                                cudaStream_t st);
+cudaError_t launch_probe_mask(const Geo& g, const int* k_per_head, const float* pq, const float* pk,
+                              uint32_t* mask_bits, uint16_t* kv_idx, int32_t* kv_cnt, cudaStream_t st);
 
 namespace {
 
@@ -76,6 +82,30 @@ int k_density(int B, double d) {
 bool tc_supported(const Geo& g) { return g.b == 64 || g.b == 128; }
 
 bool aligned1024(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 1023u) == 0; }
+
+// Per-head block budgets: k = floor(B (1 - rho)) for every head, or k_h from the per-head
+// densities, whose sum must be the layer budget H (1 - rho).
+bsa_status head_budgets_k(const Geo& g, double rho, const double* head_density, int* k) {
+    if (!(rho >= 0.0 && rho <= 1.0)) return BSA_ERR_INVALID_ARG;
+    if (head_density == nullptr) {
+        const int kk = k_rho(g.B, rho);
+        for (int h = 0; h < g.H; ++h) k[h] = kk;
+        return BSA_OK;
+    }
+    double sum = 0.0;
+    for (int h = 0; h < g.H; ++h) {
+        if (!(head_density[h] >= 0.0 && head_density[h] <= 1.0)) return BSA_ERR_INVALID_ARG;
+        sum += head_density[h];
+        k[h] = k_density(g.B, head_density[h]);
+    }
+    if (std::fabs(sum - g.H * (1.0 - rho)) > 1e-9 * g.H) return BSA_ERR_INVALID_ARG;
+    return BSA_OK;
+}
+
+// Output buffers of a block selector: the lists, counts and optional bits.
+bool lists_ok(const uint16_t* kv_idx, const int32_t* kv_cnt, const uint32_t* mask_bits) {
+    return kv_idx && kv_cnt && aligned16(kv_idx) && aligned16(kv_cnt) && (!mask_bits || aligned16(mask_bits));
+}
 
 bsa_status check_ws(const Geo& g, const void* ws, size_t bytes) {
     if (ws == nullptr || !aligned1024(ws)) return BSA_ERR_INVALID_ARG;
@@ -248,24 +278,53 @@ bsa_status bsa_predict_mask(const bsa_layout* layout, const float* pq, const flo
     if (!aligned16(pq) || !aligned16(pk) || !aligned16(kv_idx) || !aligned16(kv_cnt) ||
         (mask_bits && !aligned16(mask_bits)))
         return BSA_ERR_INVALID_ARG;
-    if (!(rho >= 0.0 && rho <= 1.0) || !(tau >= 0.0 && tau <= 1.0)) return BSA_ERR_INVALID_ARG;
+    if (!(tau >= 0.0 && tau <= 1.0)) return BSA_ERR_INVALID_ARG;
     if (g.B > 65535) return BSA_ERR_UNSUPPORTED;
     MaskParams mp;
     mp.tau = tau;
-    if (head_density == nullptr) {
-        const int k = k_rho(g.B, rho);
-        for (int h = 0; h < g.H; ++h) mp.k[h] = k;
-    } else {
-        double sum = 0.0;
-        for (int h = 0; h < g.H; ++h) {
-            if (!(head_density[h] >= 0.0 && head_density[h] <= 1.0)) return BSA_ERR_INVALID_ARG;
-            sum += head_density[h];
-            mp.k[h] = k_density(g.B, head_density[h]);
-        }
-        if (std::fabs(sum - g.H * (1.0 - rho)) > 1e-9 * g.H) return BSA_ERR_INVALID_ARG;
-    }
+    if ((s = head_budgets_k(g, rho, head_density, mp.k)) != BSA_OK) return s;
     return from_cuda(launch_mask(g, mp, pq, pk, mask_bits, kv_idx, kv_cnt, status_dev,
                                  reinterpret_cast<cudaStream_t>(stream)));
+}
+
+bsa_status bsa_random_mask(const bsa_layout* layout, double rho, const double* head_density, uint64_t seed,
+                           uint32_t* mask_bits, uint16_t* kv_idx, int32_t* kv_cnt, int32_t* status_dev,
+                           bsa_stream_t stream) {
+    (void)status_dev;
+    Geo g;
+    bsa_status s = make_geo(layout, &g);
+    if (s != BSA_OK) return s;
+    if (!lists_ok(kv_idx, kv_cnt, mask_bits)) return BSA_ERR_INVALID_ARG;
+    if (g.B > 65535) return BSA_ERR_UNSUPPORTED;
+    int k[BSA_MAX_HEADS];
+    if ((s = head_budgets_k(g, rho, head_density, k)) != BSA_OK) return s;
+    return from_cuda(launch_random_mask(g, k, seed, mask_bits, kv_idx, kv_cnt, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+bsa_status bsa_uniform_mask(const bsa_layout* layout, int32_t stride, uint32_t* mask_bits, uint16_t* kv_idx,
+                            int32_t* kv_cnt, int32_t* status_dev, bsa_stream_t stream) {
+    (void)status_dev;
+    Geo g;
+    bsa_status s = make_geo(layout, &g);
+    if (s != BSA_OK) return s;
+    if (stride < 1 || !lists_ok(kv_idx, kv_cnt, mask_bits)) return BSA_ERR_INVALID_ARG;
+    if (g.B > 65535) return BSA_ERR_UNSUPPORTED;
+    return from_cuda(launch_uniform_mask(g, stride, mask_bits, kv_idx, kv_cnt, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+bsa_status bsa_probe_mask(const bsa_layout* layout, const float* pq, const float* pk, double rho,
+                          const double* head_density, uint32_t* mask_bits, uint16_t* kv_idx, int32_t* kv_cnt,
+                          int32_t* status_dev, bsa_stream_t stream) {
+    (void)status_dev;
+    Geo g;
+    bsa_status s = make_geo(layout, &g);
+    if (s != BSA_OK) return s;
+    if (!pq || !pk || !aligned16(pq) || !aligned16(pk) || !lists_ok(kv_idx, kv_cnt, mask_bits))
+        return BSA_ERR_INVALID_ARG;
+    if (g.B > 65535) return BSA_ERR_UNSUPPORTED;
+    int k[BSA_MAX_HEADS];
+    if ((s = head_budgets_k(g, rho, head_density, k)) != BSA_OK) return s;
+    return from_cuda(launch_probe_mask(g, k, pq, pk, mask_bits, kv_idx, kv_cnt, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 bsa_status bsa_block_sparse_attn(const bsa_layout* layout, const void* q, const void* k,

@@ -36,11 +36,20 @@ class Buffers:
 class BlockSparseLayer:
     """One global-attention layer of fixed geometry and selection hyper-parameters."""
 
+    SELECTORS = ("predict", "random", "uniform", "probe")
+
     def __init__(self, frames: int, tokens_per_frame: int, special_per_frame: int, heads: int,
                  head_dim: int, block: int, dtype: str, rho: float, tau: float, head_density=None,
-                 device: str | torch.device = "cuda"):
+                 device: str | torch.device = "cuda", selector: str = "predict", seed: int = 0,
+                 stride: int = 4):
+        """selector: how the kept blocks are chosen -- "predict" (pooled softmax and the dual
+        threshold), "random" (k_h blocks uniformly at random, keyed by `seed`), "uniform"
+        (every `stride`-th block) or "probe" (the k_h blocks of highest mean-query score)."""
+        if selector not in self.SELECTORS:
+            raise ValueError(f"selector must be one of {self.SELECTORS}")
         self.layout = _lib.make_layout(frames, tokens_per_frame, special_per_frame, heads, head_dim, block, dtype)
         self.dtype = dtype
+        self.selector, self.seed, self.stride = selector, int(seed), int(stride)
         self.rho, self.tau = float(rho), float(tau)
         self.head_density = None if head_density is None else [float(x) for x in head_density]
         self.device = torch.device(device)
@@ -66,18 +75,31 @@ class BlockSparseLayer:
 
     @classmethod
     def for_workload(cls, w, head_density=None, device="cuda") -> "BlockSparseLayer":
-        return cls(w.frames, w.tokens_per_frame, w.special_per_frame, w.heads, w.head_dim, w.block,
-                   w.dtype, w.rho, w.tau, head_density, device)
+        return cls(w.frames, w.tokens_per_frame, w.layer_special, w.heads, w.head_dim, w.block,
+                   w.dtype, w.rho, w.tau, head_density, device, w.selector, w.seed, w.stride)
 
     # individual steps -------------------------------------------------------------
     def predict(self, q: torch.Tensor, k: torch.Tensor, stream: int | None = None) -> None:
         st = self._stream(stream)
         b = self.buf
-        _lib.bsa_pool_qk(self.layout, q.data_ptr(), k.data_ptr(), b.pq.data_ptr(), b.pk.data_ptr(),
-                         b.status.data_ptr(), st)
-        _lib.bsa_predict_mask(self.layout, b.pq.data_ptr(), b.pk.data_ptr(), self.rho, self.tau,
-                              self.head_density, b.mask_bits.data_ptr(), b.kv_idx.data_ptr(),
-                              b.kv_cnt.data_ptr(), b.status.data_ptr(), st)
+        if self.selector in ("predict", "probe"):
+            _lib.bsa_pool_qk(self.layout, q.data_ptr(), k.data_ptr(), b.pq.data_ptr(), b.pk.data_ptr(),
+                             b.status.data_ptr(), st)
+        self._select(st)
+
+    def _select(self, st) -> None:
+        """The block selection step, from the pooled means already in pq / pk."""
+        b = self.buf
+        args = (b.mask_bits.data_ptr(), b.kv_idx.data_ptr(), b.kv_cnt.data_ptr(), b.status.data_ptr(), st)
+        if self.selector == "predict":
+            _lib.bsa_predict_mask(self.layout, b.pq.data_ptr(), b.pk.data_ptr(), self.rho, self.tau,
+                                  self.head_density, *args)
+        elif self.selector == "random":
+            _lib.bsa_random_mask(self.layout, self.rho, self.head_density, self.seed, *args)
+        elif self.selector == "uniform":
+            _lib.bsa_uniform_mask(self.layout, self.stride, *args)
+        else:
+            _lib.bsa_probe_mask(self.layout, b.pq.data_ptr(), b.pk.data_ptr(), self.rho, self.head_density, *args)
 
     def partials(self) -> Buffers:
         """The layer's buffers, with the fp32 partials of the step-by-step path allocated."""
@@ -140,11 +162,12 @@ class BlockSparseLayer:
         # packing and pooling in one pass over Q, K, V; then mask, special rows, patch rows.
         # (Running the special rows on a second stream next to the mask and the patch rows
         # was measured slower: both attention passes are compute-bound and share the SMs.)
-        _lib.bsa_pack_pool_qkv(self.layout, qp, kp, vp, self.ws_ptr, self.ws_bytes, b.pq.data_ptr(),
-                               b.pk.data_ptr(), b.status.data_ptr(), st)
-        _lib.bsa_predict_mask(self.layout, b.pq.data_ptr(), b.pk.data_ptr(), self.rho, self.tau,
-                              self.head_density, b.mask_bits.data_ptr(), b.kv_idx.data_ptr(),
-                              b.kv_cnt.data_ptr(), b.status.data_ptr(), st)
+        if self.selector in ("predict", "probe"):
+            _lib.bsa_pack_pool_qkv(self.layout, qp, kp, vp, self.ws_ptr, self.ws_bytes, b.pq.data_ptr(),
+                                   b.pk.data_ptr(), b.status.data_ptr(), st)
+        else:   # the selection reads no pooled means
+            _lib.bsa_pack_qkv(self.layout, qp, kp, vp, self.ws_ptr, self.ws_bytes, b.status.data_ptr(), st)
+        self._select(st)
         _lib.bsa_special_dense(self.layout, qp, kp, vp, self.ws_ptr, self.ws_bytes, o.data_ptr(),
                                None, None, b.status.data_ptr(), st)
         main = None
