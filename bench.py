@@ -316,10 +316,13 @@ def _oracle_layer_sample(oracle, w, x, budget_s, seed):
 
 
 def reference_arm(args, w):
-    x = synth.make_inputs(w)
+    x = synth.make_inputs(w) if w.kind == "global" else None
     times = []
     for s in range(args.warmup + args.steps):
-        ms, threads, host_cpus, sample = oracle_layer_sample(w, x, budget_s=args.ref_budget, seed=s)
+        if w.kind == "global":
+            ms, threads, host_cpus, sample = oracle_layer_sample(w, x, budget_s=args.ref_budget, seed=s)
+        else:
+            ms, threads, host_cpus, sample = oracle_block_sample(w, budget_s=args.ref_budget, seed=s)
         if s >= args.warmup:
             times.append(ms)
     v = float(np.mean(times))
@@ -341,6 +344,15 @@ SELECTOR_TEXT = {
 }
 
 
+KIND_TEXT = {
+    "global": "",
+    "frame": "; frame-wise dense attention over each frame's {T} tokens (no mask: rho, tau, b unused)",
+    "block": "; QKV projection (C = {C} -> 3C) + this global layer + output projection, random-init weights",
+    "frame_block": "; QKV projection (C = {C} -> 3C) + frame-wise dense attention + output projection, "
+                   "random-init weights",
+}
+
+
 def workload_config(w):
     return {"workload": f"{w.name}: {w.frames} frames x ({w.patch_per_frame} patch + {w.special_per_frame} special)"
                         f" tokens, {w.heads} heads, d={w.head_dim}, b={w.block}, rho={w.rho}, tau={w.tau}"
@@ -348,7 +360,8 @@ def workload_config(w):
                            if w.head_budgets else "")
                         + SELECTOR_TEXT[w.selector].format(seed=w.seed, stride=w.stride)
                         + (", special tokens read as patch tokens (no dense special path)"
-                           if w.sparse_specials else ""),
+                           if w.sparse_specials else "")
+                        + KIND_TEXT[w.kind].format(T=w.tokens_per_frame, C=w.heads * w.head_dim),
             "frames": w.frames, "tokens_per_frame": w.tokens_per_frame, "heads": w.heads, "head_dim": w.head_dim,
             "block": w.block, "rho": w.rho, "tau": w.tau, "global_batch": 1, "seq_len": w.n_tokens,
             "parallelism": "replicas",
@@ -405,6 +418,199 @@ def e2e_pipelined(torch, L, q, k, v, steps: int, path: str) -> float:
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     run(steps, t0, t1)
     return t0.elapsed_time(t1) / steps
+
+
+# ---------------------------------------------------------------------------- frame / block steps
+def oracle_block_sample(w, budget_s: float, seed: int = 7):
+    """Times the fp64 oracle of a frame-attention or projection-block step on bounded samples
+    and scales each part to one step: the projections on seeded token rows, the frame attention
+    on seeded (row, head) pairs, the global layer through oracle_layer_sample."""
+    import oracle  # noqa: F401
+    from oracle import layer_io
+    from threadpoolctl import threadpool_info, threadpool_limits
+    host_cpus = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    g = np.random.default_rng(seed)
+    N, H, d = w.n_tokens, w.heads, w.head_dim
+    C = H * d
+    parts, est = [], 0.0
+    with threadpool_limits(limits=host_cpus):
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        if w.kind in ("block", "frame_block"):
+            bi = synth.make_block_inputs(w.with_(frames=1))          # weights do not depend on F
+            rows = min(N, 4096)
+            X = g.standard_normal((rows, C))
+            t0 = time.perf_counter()
+            layer_io.qkv_project(X, synth.decode(bi.w_qkv, "bf16"), bi.b_qkv, H, d)
+            layer_io.out_project(X.reshape(rows, H, d), synth.decode(bi.w_o, "bf16"), bi.b_o)
+            t = time.perf_counter() - t0
+            est += t * N / rows
+            parts.append(f"projections of {rows}/{N} token rows ({t:.1f} s)")
+        if w.kind in ("frame", "frame_block"):
+            x = synth.make_inputs(w.with_(frames=min(w.frames, 4)))
+            Q, K, V = (synth.decode(a, "bf16") for a in (x.q, x.k, x.v))
+            t0, done = time.perf_counter(), 0
+            while time.perf_counter() - t0 < budget_s * 0.5:
+                rows = g.integers(0, len(Q), 256)
+                heads = g.integers(0, H, 256)
+                layer_io.frame_attention_rows(Q, K, V, w.tokens_per_frame, rows, heads)
+                done += 256
+            t = time.perf_counter() - t0
+            est += t * N * H / done
+            parts.append(f"frame attention of {done}/{N * H} (row, head) pairs ({t:.1f} s)")
+        if w.kind == "block":
+            ms, _, _, sample = oracle_layer_sample(w.with_(kind="global"), synth.make_inputs(w), budget_s * 0.5, seed)
+            est += ms / 1e3
+            parts.append("global layer: " + sample)
+    return est * 1e3, threads, host_cpus, "sampled estimate: " + "; ".join(parts) + "; each scaled to one step"
+
+
+def block_stage_calls(w, L, tensors, status, sp):
+    """(stage, callable, launches) of one frame-attention or projection-block step."""
+    from view_transformers_b200 import _lib
+    lay = _lib.layout_of(w)
+    t = tensors
+    ptr = (lambda a: 0 if a is None else a.data_ptr())
+    calls = []
+    if w.kind in ("block", "frame_block"):
+        calls.append(("qkv", lambda: _lib.bsa_qkv_project(lay, t["x"].data_ptr(), t["w_qkv"].data_ptr(),
+                                                          ptr(t["b_qkv"]), t["q"].data_ptr(), t["k"].data_ptr(),
+                                                          t["v"].data_ptr(), status, sp), 1))
+    if w.kind in ("frame", "frame_block"):
+        calls.append(("pack_frames", lambda: _lib.bsa_pack_frames(lay, t["q"].data_ptr(), t["k"].data_ptr(),
+                                                                  t["v"].data_ptr(), t["ws"], t["ws_bytes"], status,
+                                                                  sp), 1))
+        calls.append(("frame_attn", lambda: _lib.bsa_frame_attention(lay, t["ws"], t["ws_bytes"], t["o"].data_ptr(),
+                                                                     status, sp), 1))
+    else:
+        calls.append(("global_layer", lambda: L.forward(t["q"], t["k"], t["v"], stream=sp, out=t["o"]), 5))
+    if w.kind in ("block", "frame_block"):
+        calls.append(("out", lambda: _lib.bsa_out_project(lay, t["o"].data_ptr(), t["w_o"].data_ptr(), ptr(t["b_o"]),
+                                                          t["y"].data_ptr(), status, sp), 1))
+    return calls
+
+
+def bench_block(args, w, world, rank, local, dist):
+    """One step = the frame-wise attention layer, or a whole block (QKV projection, attention,
+    output projection), on synthetic tokens and random-init weights resident in HBM."""
+    import torch
+    from view_transformers_b200 import _lib, layer
+    N, H, d = w.n_tokens, w.heads, w.head_dim
+    C = H * d
+    dev = torch.device("cuda", local)
+    x = synth.make_inputs(w)
+    t = {k_: layer.to_device(a, "bf16") for k_, a in (("q", x.q), ("k", x.k), ("v", x.v))}
+    t["o"] = torch.empty_like(t["q"])
+    L = None
+    if w.kind in ("block", "frame_block"):
+        bi = synth.make_block_inputs(w)
+        t["x"] = layer.to_device(bi.x, "bf16")
+        t["w_qkv"], t["w_o"] = layer.to_device(bi.w_qkv, "bf16"), layer.to_device(bi.w_o, "bf16")
+        t["b_qkv"], t["b_o"] = torch.from_numpy(bi.b_qkv).to(dev), torch.from_numpy(bi.b_o).to(dev)
+        t["y"] = torch.empty((N, C), dtype=torch.bfloat16, device=dev)
+    if w.kind in ("frame", "frame_block"):
+        nbytes = _lib.bsa_frame_workspace_size(_lib.layout_of(w))
+        t["ws_buf"] = torch.empty(nbytes + 1024, dtype=torch.uint8, device=dev)
+        t["ws"], t["ws_bytes"] = (t["ws_buf"].data_ptr() + 1023) // 1024 * 1024, nbytes
+    else:
+        dens = _lib.bsa_head_budgets(x.scores, w.rho, 1.0) if x.scores is not None else None
+        L = layer.BlockSparseLayer.for_workload(w.with_(kind="global"), head_density=dens)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    sp = torch.cuda.current_stream().cuda_stream
+    calls = block_stage_calls(w, L, t, status.data_ptr(), sp)
+
+    def run(steps, stage_ms=None):
+        st = torch.cuda.current_stream()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(steps)]
+        for s in range(steps):
+            evs[s][0].record(st)
+            for i, (_, fn, _) in enumerate(calls):
+                fn()
+                evs[s][i + 1].record(st)
+        torch.cuda.synchronize()
+        if stage_ms is not None:
+            for i, (name, _, _) in enumerate(calls):
+                stage_ms[name] = float(np.mean([evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(steps)]))
+        return evs[0][0].elapsed_time(evs[-1][-1])
+
+    run(args.warmup)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    stage_ms = {}
+    with ClockSampler(local) as clk:
+        total_ms = run(args.steps, stage_ms)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    code = _lib.bsa_check_status(status.data_ptr(), sp) or (L.check_status() if L is not None else 0)
+    clocks = clk.summary()
+    total_ms = max_over_ranks(total_ms, dist, "cuda")
+    ms_per_step = total_ms / args.steps
+    value = job_ms_per_layer(total_ms, args.steps, world)
+
+    # algorithmic work per stage
+    flops = {"qkv": 2.0 * N * C * 3 * C, "out": 2.0 * N * C * C,
+             "frame_attn": 4.0 * d * H * w.frames * float(w.tokens_per_frame) ** 2}
+    if L is not None:
+        kv_cnt = L.buf.kv_cnt.cpu().numpy()
+        kv_idx = L.buf.kv_idx.cpu().numpy().view(np.uint16)
+        flops["global_layer"] = sparse_flops(kv_cnt, kv_idx, w) + special_flops(w)
+    hbm, tf_burst, tf_sus, peak_src = peaks()
+    tflops = {k_: flops[k_] / (stage_ms[k_] * 1e-3) / 1e12 for k_ in stage_ms if k_ in flops}
+    dom = max((k_ for k_ in stage_ms if k_ in flops), key=lambda k_: stage_ms[k_])
+    kernel_name = {"qkv": "bsa_qkv_project (tcgen05 GEMM)", "out": "bsa_out_project (tcgen05 GEMM)",
+                   "frame_attn": "bsa_frame_attention (tcgen05 attention)",
+                   "global_layer": "global layer (five launches, fused tcgen05 attention dominant)"}[dom]
+
+    # end to end: the step's inputs from pinned host memory, its output back, every step
+    ins = ["x"] if "x" in t else ["q", "k", "v"]
+    outk = "y" if "y" in t else "o"
+    host_in = {k_: t[k_].cpu().pin_memory() for k_ in ins}
+    host_out = torch.empty(t[outk].shape, dtype=t[outk].dtype).pin_memory()
+    e2e_ms = float("nan")
+    if args.e2e_steps > 0:
+        def e2e(n):
+            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(n):
+                for k_ in ins:
+                    t[k_].copy_(host_in[k_], non_blocking=True)
+                for _, fn, _ in calls:
+                    fn()
+                host_out.copy_(t[outk], non_blocking=True)
+            b_.record()
+            torch.cuda.synchronize()
+            return a.elapsed_time(b_) / n
+        e2e(2)
+        e2e_ms = e2e(min(args.e2e_steps, 10))
+    e2e_value = max_over_ranks(e2e_ms, dist, "cuda") / world
+    h2d = sum(host_in[k_].numel() * host_in[k_].element_size() for k_ in ins)
+    d2h = host_out.numel() * host_out.element_size()
+    achieved = tflops[dom]
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic (seeded N(0,1) tokens / Q, K, V; random-init projection weights N(0, 1/C))",
+        "config": workload_config(w),
+        "stage_ms": stage_ms, "stage_tflops": tflops, "step_flops": sum(flops[k_] for k_ in stage_ms if k_ in flops),
+        "roofline": {"kernel": kernel_name, "bound": "tensor", "achieved": achieved, "peak": tf_burst,
+                     "unit": "TFLOP/s", "frac": achieved / tf_burst,
+                     "peak_kind": f"{peak_src} burst bf16", "frac_of_sustained": achieved / tf_sus,
+                     "flops_per_launch": flops[dom], "launch_ms": stage_ms[dom], "traffic": None},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "copies": "pinned host buffers, copies on the compute stream (not overlapped)"},
+        "gpu_launches": sum(c[2] for c in calls) * args.steps,
+        "clocks": clocks, "device_status": code,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        ms, threads, host_cpus, sample = oracle_block_sample(w, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": ms, "unit": UNIT, "cores": threads, "host_cpus": host_cpus,
+                                "kind": "oracle", "extrapolated": True, "sample": sample}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.destroy_process_group()
 
 
 # ---------------------------------------------------------------------------- ranks
@@ -465,6 +671,8 @@ def main():
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
 
+    if w.kind != "global":
+        return bench_block(args, w, world, rank, local, dist)
     path = args.path or ("fused" if w.dtype == "bf16" else "five")
     x = synth.make_inputs(w)
     density = _lib.bsa_head_budgets(x.scores, w.rho, 1.0) if x.scores is not None else None

@@ -254,6 +254,46 @@ BSA_API bsa_status bsa_block_sparse_attn_fused(const bsa_layout* layout, const v
                                                int32_t* status_dev, bsa_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
+ * The steps on either side of the layer. The pages put the global attention inside an
+ * aggregator that alternates frame-wise and global multi-head attention ("Block-Sparse Global
+ * Attention for Efficient Multi-View Geometry Transformers", 研究背景: 交替「帧内注意力 + 全局
+ * 注意力」; "SAF3R: Dynamic Sparse Attention for Feed-Forward 3D Reconstruction Transformers",
+ * 图2). bf16 layouts only (BSA_ERR_UNSUPPORTED otherwise); fp32 accumulation, bf16 results
+ * rounded to nearest even. C = heads * head_dim channels.
+ *
+ * QKV projection: [q | k | v] = x W_qkv^T + b_qkv, channel c of each third = head c / d,
+ * dimension c % d (the usual multi-head split); written as three [N, H, d] tensors.
+ *   x      : device, bf16 [N, C] (row stride C)
+ *   w_qkv  : device, bf16 [3C, C] (output features x input features, row-major)
+ *   b_qkv  : device, float32 [3C], or NULL for no bias
+ *   q, k, v: device, bf16 [N, H, d] each
+ * tcgen05 MMA (128 x 256 output tiles, TMEM accumulators, TMA operand tiles). */
+BSA_API bsa_status bsa_qkv_project(const bsa_layout* layout, const void* x, const void* w_qkv, const float* b_qkv,
+                                   void* q, void* k, void* v, int32_t* status_dev, bsa_stream_t stream);
+
+/* Output projection: y = o W_o^T + b_o with o's heads concatenated ([N, H, d] read as [N, C]).
+ *   o   : device, bf16 [N, H, d];  w_o : device, bf16 [C, C];  b_o : device, float32 [C] or NULL
+ *   y   : device, bf16 [N, C] (must not overlap o) */
+BSA_API bsa_status bsa_out_project(const bsa_layout* layout, const void* o, const void* w_o, const float* b_o,
+                                   void* y, int32_t* status_dev, bsa_stream_t stream);
+
+/* Frame-wise attention, two calls. bsa_pack_frames copies Q, K and V per (head, frame) into
+ * the workspace: the frame's T tokens, special tokens included, padded with zero rows to a
+ * multiple of 128 (V as fp16, range-checked as in bsa_pack_qkv). bsa_frame_attention then
+ * lets every token attend densely (Eq. (1)) over the T tokens of its own frame on the tensor
+ * cores, reading only the workspace, and writes every row of out.
+ *   q, k, v, out : device, bf16 [N, H, d]
+ *   workspace    : device, at least bsa_frame_workspace_size() bytes, 1024-byte aligned */
+BSA_API bsa_status bsa_pack_frames(const bsa_layout* layout, const void* q, const void* k, const void* v,
+                                   void* workspace, size_t workspace_bytes, int32_t* status_dev,
+                                   bsa_stream_t stream);
+BSA_API bsa_status bsa_frame_attention(const bsa_layout* layout, const void* workspace, size_t workspace_bytes,
+                                       void* out, int32_t* status_dev, bsa_stream_t stream);
+/* Bytes of the frame-wise attention's workspace: 3 H F ceil(T / 128) 128 rows of 128 bytes
+ * (0 for f32 layouts). */
+BSA_API bsa_status bsa_frame_workspace_size(const bsa_layout* layout, size_t* bytes);
+
+/* ---------------------------------------------------------------------------------
  * Allocation-free attention (bf16). The pages have no counterpart: this entry point
  * exists for callers that cannot allocate device memory -- code running under a host
  * framework whose memory pool owns every device allocation, or latency-critical loops in

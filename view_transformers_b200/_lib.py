@@ -44,6 +44,11 @@ _SIGS = {
     "bsa_merge": [_LP, _vp, _vp, _vp, _vp, _vp, _i32p, _st],
     "bsa_block_sparse_attn_fused": [_LP, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp, _i32p, _st],
     "bsa_attention_noalloc": [_LP, _vp, _vp, _vp, _vp, _vp, _vp, _i32p, _st],
+    "bsa_qkv_project": [_LP, _vp, _vp, _vp, _vp, _vp, _vp, _i32p, _st],
+    "bsa_out_project": [_LP, _vp, _vp, _vp, _vp, _i32p, _st],
+    "bsa_pack_frames": [_LP, _vp, _vp, _vp, _vp, _sz, _i32p, _st],
+    "bsa_frame_attention": [_LP, _vp, _sz, _vp, _i32p, _st],
+    "bsa_frame_workspace_size": [_LP, ctypes.POINTER(ctypes.c_size_t)],
     "bsa_random_mask": [_LP, ctypes.c_double, ctypes.c_void_p, ctypes.c_uint64, _vp, _vp, _vp, _i32p, _st],
     "bsa_uniform_mask": [_LP, ctypes.c_int32, _vp, _vp, _vp, _i32p, _st],
     "bsa_probe_mask": [_LP, _vp, _vp, ctypes.c_double, ctypes.c_void_p, _vp, _vp, _vp, _i32p, _st],
@@ -214,6 +219,30 @@ def bsa_block_sparse_attn_fused(layout, q, k, v, workspace, workspace_bytes, kv_
                                 stream=0) -> None:
     _check("bsa_block_sparse_attn_fused", load().bsa_block_sparse_attn_fused(
         ctypes.byref(layout), q, k, v, workspace, workspace_bytes, kv_idx, kv_cnt, out, status, stream))
+
+
+def bsa_qkv_project(layout, x, w_qkv, b_qkv, q, k, v, status=0, stream=0) -> None:
+    _check("bsa_qkv_project", load().bsa_qkv_project(ctypes.byref(layout), x, w_qkv, b_qkv, q, k, v, status, stream))
+
+
+def bsa_out_project(layout, o, w_o, b_o, y, status=0, stream=0) -> None:
+    _check("bsa_out_project", load().bsa_out_project(ctypes.byref(layout), o, w_o, b_o, y, status, stream))
+
+
+def bsa_frame_workspace_size(layout) -> int:
+    out = ctypes.c_size_t()
+    _check("bsa_frame_workspace_size", load().bsa_frame_workspace_size(ctypes.byref(layout), ctypes.byref(out)))
+    return out.value
+
+
+def bsa_pack_frames(layout, q, k, v, workspace, workspace_bytes, status=0, stream=0) -> None:
+    _check("bsa_pack_frames", load().bsa_pack_frames(ctypes.byref(layout), q, k, v, workspace, workspace_bytes,
+                                                     status, stream))
+
+
+def bsa_frame_attention(layout, workspace, workspace_bytes, out, status=0, stream=0) -> None:
+    _check("bsa_frame_attention", load().bsa_frame_attention(ctypes.byref(layout), workspace, workspace_bytes, out,
+                                                             status, stream))
 
 
 def bsa_attention_noalloc(layout, q, k, v, kv_idx, kv_cnt, out, status=0, stream=0) -> None:

@@ -37,6 +37,10 @@ class Workload:
     # the ablation without the dense special path: the layer reads the S special tokens of
     # every frame as patch tokens (pooled and sparsified with them)
     sparse_specials: bool = False
+    # what one step runs: "global" (the block-sparse global attention layer), "frame" (the
+    # frame-wise dense attention), "block" / "frame_block" (that attention between the QKV and
+    # output projections, from tokens x [N, C] to y [N, C])
+    kind: str = "global"
 
     @property
     def layer_special(self) -> int:
@@ -105,6 +109,14 @@ RANDOM_NOSPECIAL100 = PERHEAD100.with_(name="random_nospecial100", selector="ran
 UNIFORM100 = PERHEAD100.with_(name="uniform100", selector="uniform", stride=4, head_budgets=False)
 PROBE100 = PERHEAD100.with_(name="probe100", selector="probe")
 
-ALL = {w.name: w for w in (TINY, VGGT518, SWEEP_R50, SWEEP_R75, SWEEP_R90, PERHEAD100,
+# The steps on either side of the layer ("Block-Sparse Global Attention...", 研究背景: the
+# aggregator alternates frame-wise and global attention; "SAF3R...", 图2): frame-wise dense
+# attention over the 782 tokens of each frame as a second workload, and whole blocks with the
+# QKV and output projections (random-init weights).
+FRAME100 = PERHEAD100.with_(name="frame100", kind="frame", head_budgets=False)
+BLOCK100 = PERHEAD100.with_(name="block100", kind="block")
+FRAME_BLOCK100 = PERHEAD100.with_(name="frame_block100", kind="frame_block", head_budgets=False)
+
+ALL = {w.name: w for w in (FRAME100, BLOCK100, FRAME_BLOCK100, TINY, VGGT518, SWEEP_R50, SWEEP_R75, SWEEP_R90, PERHEAD100,
                            PERHEAD100_TAU95, LONG500, TINY_TAU0, SWEEP_TAU0, CDF_ONLY100, NOSPECIAL100,
                            RANDOM100, RANDOM_NOSPECIAL100, UNIFORM100, PROBE100)}

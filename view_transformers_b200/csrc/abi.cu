@@ -36,6 +36,11 @@ cudaError_t launch_uniform_mask(const Geo& g, int stride, uint32_t* mask_bits, u
                                 cudaStream_t st);
 cudaError_t launch_probe_mask(const Geo& g, const int* k_per_head, const float* pq, const float* pk,
                               uint32_t* mask_bits, uint16_t* kv_idx, int32_t* kv_cnt, cudaStream_t st);
+cudaError_t launch_gemm_bf16(int M, int N, int K, const void* a, const void* b, const float* bias,
+                             void* const out[3], int split, int32_t* status, cudaStream_t st);
+cudaError_t launch_pack_frames(const Geo& g, const void* q, const void* k, const void* v, void* ws,
+                               int32_t* status, cudaStream_t st);
+cudaError_t launch_attn_frame(const Geo& g, const void* ws, void* out, int32_t* status, cudaStream_t st);
 
 namespace {
 
@@ -399,6 +404,69 @@ bsa_status bsa_block_sparse_attn_fused(const bsa_layout* layout, const void* q, 
     if (s != BSA_OK) return s;
     return from_cuda(launch_attn_tc(g, 3, workspace, kv_idx, kv_cnt, nullptr, nullptr, out, status_dev,
                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
+bsa_status bsa_qkv_project(const bsa_layout* layout, const void* x, const void* w_qkv, const float* b_qkv,
+                           void* q, void* k, void* v, int32_t* status_dev, bsa_stream_t stream) {
+    Geo g;
+    bsa_status s = make_geo(layout, &g);
+    if (s != BSA_OK) return s;
+    if (layout->dtype != BSA_BF16) return BSA_ERR_UNSUPPORTED;
+    if (!x || !w_qkv || !q || !k || !v) return BSA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_qkv) || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+        (b_qkv && !aligned16(b_qkv)))
+        return BSA_ERR_INVALID_ARG;
+    const int C = g.H * g.d;
+    void* const outs[3] = {q, k, v};
+    return from_cuda(launch_gemm_bf16(g.N, 3 * C, C, x, w_qkv, b_qkv, outs, C, status_dev,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+bsa_status bsa_out_project(const bsa_layout* layout, const void* o, const void* w_o, const float* b_o, void* y,
+                           int32_t* status_dev, bsa_stream_t stream) {
+    Geo g;
+    bsa_status s = make_geo(layout, &g);
+    if (s != BSA_OK) return s;
+    if (layout->dtype != BSA_BF16) return BSA_ERR_UNSUPPORTED;
+    if (!o || !w_o || !y || !aligned16(o) || !aligned16(w_o) || !aligned16(y) || (b_o && !aligned16(b_o)))
+        return BSA_ERR_INVALID_ARG;
+    const int C = g.H * g.d;
+    void* const outs[3] = {y, y, y};
+    return from_cuda(launch_gemm_bf16(g.N, C, C, o, w_o, b_o, outs, C, status_dev,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+bsa_status bsa_frame_workspace_size(const bsa_layout* layout, size_t* bytes) {
+    if (bytes == nullptr) return BSA_ERR_INVALID_ARG;
+    Geo g;
+    const bsa_status s = make_geo(layout, &g);
+    if (s != BSA_OK) return s;
+    *bytes = layout->dtype == BSA_BF16 ? frame_layout(g).bytes : 0;
+    return BSA_OK;
+}
+
+bsa_status bsa_pack_frames(const bsa_layout* layout, const void* q, const void* k, const void* v,
+                           void* workspace, size_t workspace_bytes, int32_t* status_dev, bsa_stream_t stream) {
+    Geo g;
+    bsa_status s = make_geo(layout, &g);
+    if (s != BSA_OK) return s;
+    if (layout->dtype != BSA_BF16) return BSA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !aligned16(q) || !aligned16(k) || !aligned16(v)) return BSA_ERR_INVALID_ARG;
+    if (workspace == nullptr || !aligned1024(workspace) || workspace_bytes < frame_layout(g).bytes)
+        return BSA_ERR_INVALID_ARG;
+    return from_cuda(launch_pack_frames(g, q, k, v, workspace, status_dev, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+bsa_status bsa_frame_attention(const bsa_layout* layout, const void* workspace, size_t workspace_bytes, void* out,
+                               int32_t* status_dev, bsa_stream_t stream) {
+    Geo g;
+    bsa_status s = make_geo(layout, &g);
+    if (s != BSA_OK) return s;
+    if (layout->dtype != BSA_BF16) return BSA_ERR_UNSUPPORTED;
+    if (!out || !aligned16(out)) return BSA_ERR_INVALID_ARG;
+    if (workspace == nullptr || !aligned1024(workspace) || workspace_bytes < frame_layout(g).bytes)
+        return BSA_ERR_INVALID_ARG;
+    return from_cuda(launch_attn_frame(g, workspace, out, status_dev, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 bsa_status bsa_merge(const bsa_layout* layout, const float* o_pp, const float* lse_pp,

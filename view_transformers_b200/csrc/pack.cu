@@ -196,7 +196,50 @@ pack_pool_kernel(Geo g, PackedLayout pl, const __nv_bfloat16* __restrict__ q,
     }
     if (out_of_range) record_error(status, BSA_ERR_RANGE);
 }
+// Per-frame packing for the frame-wise attention (frame_layout): every token of frame f,
+// special tokens included, goes to row r of the (head, frame) slab; rows T .. t_pad-1 are
+// zero. Thread order follows the token rows of the input (2 KB of one token per 128 threads
+// at 16 heads), so reads are contiguous.
+__global__ void __launch_bounds__(256)
+pack_frames_kernel(Geo g, FrameLayout fl, const __nv_bfloat16* __restrict__ q,
+                   const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+                   unsigned char* __restrict__ ws, int32_t* status) {
+    bool out_of_range = false;
+    const int chunks = g.H * 8;
+    const size_t total = (size_t)g.F * fl.t_pad * chunks;
+    for (size_t x = blockIdx.x * (size_t)blockDim.x + threadIdx.x; x < total;
+         x += (size_t)gridDim.x * blockDim.x) {
+        const size_t fr = x / chunks;                       // (frame, row) pair
+        const int c = (int)(x - fr * chunks);
+        const int h = c >> 3, c8 = c & 7;
+        const int f = (int)(fr / fl.t_pad);
+        const int r = (int)(fr - (size_t)f * fl.t_pad);
+        uint4 vq = make_uint4(0, 0, 0, 0), vk = vq, vv = vq;
+        if (r < g.T) {
+            const size_t off = ((size_t)f * g.T + r) * g.H * 64 + (size_t)h * 64 + c8 * 8;
+            vq = __ldg(reinterpret_cast<const uint4*>(q + off));
+            vk = __ldg(reinterpret_cast<const uint4*>(k + off));
+            const uint4 w = __ldg(reinterpret_cast<const uint4*>(v + off));
+            out_of_range |= beyond_f16(w);
+            vv = bf16x8_to_f16x8(w);
+        }
+        const size_t dst = (((size_t)h * g.F + f) * fl.t_pad + r) * 128 + c8 * 16;
+        *reinterpret_cast<uint4*>(ws + fl.qf + dst) = vq;
+        *reinterpret_cast<uint4*>(ws + fl.kf + dst) = vk;
+        *reinterpret_cast<uint4*>(ws + fl.vf + dst) = vv;
+    }
+    if (out_of_range) record_error(status, BSA_ERR_RANGE);
+}
 }  // namespace
+
+cudaError_t launch_pack_frames(const Geo& g, const void* q, const void* k, const void* v, void* ws,
+                               int32_t* status, cudaStream_t st) {
+    pack_frames_kernel<<<num_sms() * 8, 256, 0, st>>>(g, frame_layout(g), static_cast<const __nv_bfloat16*>(q),
+                                                      static_cast<const __nv_bfloat16*>(k),
+                                                      static_cast<const __nv_bfloat16*>(v),
+                                                      static_cast<unsigned char*>(ws), status);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_pack(const Geo& g, const void* q, const void* k, const void* v, void* ws,
                         int32_t* status, cudaStream_t st) {

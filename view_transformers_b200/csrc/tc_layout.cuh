@@ -63,4 +63,23 @@ __host__ __device__ inline PackedLayout packed_layout(const Geo& g) {
     return pl;
 }
 
+// Per-frame packing for the frame-wise attention: per head and frame, the frame's T tokens
+// (special tokens included) padded with zero rows to a multiple of 128; Q, K bf16, V fp16.
+struct FrameLayout {
+    int t_pad;           // rows per (head, frame)
+    size_t qf, kf, vf;   // byte offsets of [H][F][t_pad][64]
+    size_t bytes;
+};
+
+__host__ __device__ inline FrameLayout frame_layout(const Geo& g) {
+    FrameLayout fl;
+    fl.t_pad = (g.T + 127) / 128 * 128;
+    const size_t one = (size_t)g.H * g.F * fl.t_pad * 128;
+    fl.qf = 0;
+    fl.kf = one;
+    fl.vf = 2 * one;
+    fl.bytes = 3 * one;
+    return fl;
+}
+
 }  // namespace bsa

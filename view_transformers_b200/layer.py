@@ -205,6 +205,53 @@ class BlockSparseLayer:
         return bits[..., :self.B].astype(bool)
 
 
+class AttentionBlock:
+    """The projections around one attention layer of the aggregator: x [N, C] -> QKV projection
+    -> attention (global block-sparse `layer`, or frame-wise when layer is None) -> output
+    projection -> y [N, C] (bf16). Weights are device tensors: w_qkv [3C, C], b_qkv [3C] fp32 or
+    None, w_o [C, C], b_o [C] fp32 or None."""
+
+    def __init__(self, frames: int, tokens_per_frame: int, special_per_frame: int, heads: int, head_dim: int,
+                 w_qkv, b_qkv, w_o, b_o, layer: "BlockSparseLayer | None" = None, device="cuda"):
+        self.layout = _lib.make_layout(frames, tokens_per_frame, special_per_frame, heads, head_dim,
+                                       layer.layout.block if layer is not None else 128, "bf16")
+        self.w_qkv, self.b_qkv, self.w_o, self.b_o = w_qkv, b_qkv, w_o, b_o
+        self.layer = layer
+        self.device = torch.device(device)
+        N = frames * tokens_per_frame
+        shape = (N, heads, head_dim)
+        self.q, self.k, self.v, self.o = (torch.empty(shape, dtype=torch.bfloat16, device=self.device)
+                                          for _ in range(4))
+        self.y = torch.empty((N, heads * head_dim), dtype=torch.bfloat16, device=self.device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=self.device)
+        self.frame_ws_bytes = _lib.bsa_frame_workspace_size(self.layout) if layer is None else 0
+        self.frame_ws = torch.empty(self.frame_ws_bytes + 1024, dtype=torch.uint8, device=self.device)
+        self.frame_ws_ptr = (self.frame_ws.data_ptr() + 1023) // 1024 * 1024
+
+    def forward(self, x: torch.Tensor, stream: int | None = None) -> torch.Tensor:
+        st = torch.cuda.current_stream(self.device).cuda_stream if stream is None else stream
+        s = self.status.data_ptr()
+        ptr = (lambda t: 0 if t is None else t.data_ptr())
+        _lib.bsa_qkv_project(self.layout, x.data_ptr(), self.w_qkv.data_ptr(), ptr(self.b_qkv), self.q.data_ptr(),
+                             self.k.data_ptr(), self.v.data_ptr(), s, st)
+        if self.layer is None:
+            _lib.bsa_pack_frames(self.layout, self.q.data_ptr(), self.k.data_ptr(), self.v.data_ptr(),
+                                 self.frame_ws_ptr, self.frame_ws_bytes, s, st)
+            _lib.bsa_frame_attention(self.layout, self.frame_ws_ptr, self.frame_ws_bytes, self.o.data_ptr(), s, st)
+        else:
+            self.layer.forward(self.q, self.k, self.v, stream=st, out=self.o)
+        _lib.bsa_out_project(self.layout, self.o.data_ptr(), self.w_o.data_ptr(), ptr(self.b_o), self.y.data_ptr(),
+                             s, st)
+        return self.y
+
+    def check_status(self, stream: int | None = None) -> int:
+        st = torch.cuda.current_stream(self.device).cuda_stream if stream is None else stream
+        code = _lib.bsa_check_status(self.status.data_ptr(), st)
+        if self.layer is not None:
+            code = code or self.layer.check_status(stream)
+        return code
+
+
 def to_device(x, dtype: str, device="cuda") -> torch.Tensor:
     """Storage array from synth (uint16 bf16 bits or float32) -> device tensor of the layer dtype."""
     import numpy as np

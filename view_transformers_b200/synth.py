@@ -140,3 +140,34 @@ def make_inputs(w: Workload) -> LayerInputs:
 def decode(a: np.ndarray, dtype: str) -> np.ndarray:
     """Storage array (bf16 bits or float32) -> float64, exactly."""
     return _decode(a, dtype)
+
+
+@dataclass
+class BlockInputs:
+    """Synthetic inputs of one attention block: tokens x [N, C] and random-init projection
+    weights (bf16 bits), biases fp32. W ~ N(0, 1/C) keeps the projected values near unit
+    scale; biases ~ N(0, 0.02^2)."""
+    x: np.ndarray        # uint16 [N, C]
+    w_qkv: np.ndarray    # uint16 [3C, C]
+    b_qkv: np.ndarray    # float32 [3C]
+    w_o: np.ndarray      # uint16 [C, C]
+    b_o: np.ndarray      # float32 [C]
+
+
+def make_block_inputs(w: Workload) -> BlockInputs:
+    """Drawn from Generator(PCG64(SeedSequence([seed, 10 + t]))) for t = x, w_qkv, b_qkv, w_o,
+    b_o in that order, in fp64, then rounded (bf16 RNE, or fp32 for the biases)."""
+    C = w.heads * w.head_dim
+    N = w.n_tokens
+
+    def draw(t, shape, std):
+        g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([w.seed, 10 + t])))
+        return g.standard_normal(shape) * std
+
+    return BlockInputs(
+        x=f64_to_bf16_bits(draw(0, (N, C), 1.0)),
+        w_qkv=f64_to_bf16_bits(draw(1, (3 * C, C), C ** -0.5)),
+        b_qkv=draw(2, 3 * C, 0.02).astype(np.float32),
+        w_o=f64_to_bf16_bits(draw(3, (C, C), C ** -0.5)),
+        b_o=draw(4, C, 0.02).astype(np.float32),
+    )
