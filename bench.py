@@ -174,7 +174,7 @@ def step_calls(L, q, k, v, path: str):
     status = b.status.data_ptr()
     lay = L.layout
     qp, kp, vp = q.data_ptr(), k.data_ptr(), v.data_ptr()
-    mask = ("mask", lambda: L._select(sp), 1)
+    mask = ("mask", lambda: L._select(sp, v), 2 if L.selector == "ress" else 1)
     if path == "fused" and L.selector in ("random", "uniform"):   # no pooled means needed
         calls = [("pack", lambda: _lib.bsa_pack_qkv(lay, qp, kp, vp, L.ws_ptr, L.ws_bytes, status, sp), 1), mask]
     elif path == "fused":
@@ -282,8 +282,14 @@ def _oracle_layer_sample(oracle, w, x, budget_s, seed):
         selected = selectors.random_mask(lay, kh, w.seed)
     elif w.selector == "uniform":
         selected = selectors.uniform_mask(lay, w.stride)
-    else:
+    elif w.selector == "probe":
         selected = selectors.probe_mask(Q, K, lay, kh)[1]
+    else:
+        selected = None          # drift-score rows: selected per sampled pair below
+        from oracle import ress
+        PQ, PK = oracle.pool(Q, lay), oracle.pool(K, lay)
+        PV = oracle.pool(oracle.to_f64(x.v, w.dtype), lay)
+        probs = oracle.pooled_probs(PQ, PK, lay.head_dim)
     t_mask = time.perf_counter() - t0
     V = oracle.to_f64(x.v, w.dtype)
     g = np.random.default_rng(seed)
@@ -293,7 +299,9 @@ def _oracle_layer_sample(oracle, w, x, budget_s, seed):
     sr = oracle.special_rows(lay)
     for h, i in pairs:
         rows = oracle.patch_rows(lay)[slice(*oracle.block_bounds(lay, i))]
-        keys = np.concatenate([sr, oracle.patch_keys_of(lay, selected[h, i])])
+        kept = selected[h, i] if selected is not None else ress.select_row(probs[h, i], PV[h], int(kh[h]),
+                                                                          w.rounds)[0]
+        keys = np.concatenate([sr, oracle.patch_keys_of(lay, kept)])
         oracle.attend(Q[rows, h], K[keys, h], V[keys, h])
         done += 1
         if time.perf_counter() - t1 > budget_s * 0.8:
@@ -341,6 +349,7 @@ SELECTOR_TEXT = {
     "random": ", random blocks (k_h per row, Philox4x32-10 keys, seed {seed})",
     "uniform": ", fixed-stride uniform sampling (every {stride}th block)",
     "probe": ", query-probe Top-K (mean-query scores, k_h per head)",
+    "ress": ", drift-score selection (k_h per head, up to {rounds} restoration rounds)",
 }
 
 
@@ -358,7 +367,7 @@ def workload_config(w):
                         f" tokens, {w.heads} heads, d={w.head_dim}, b={w.block}, rho={w.rho}, tau={w.tau}"
                         + (", per-head budgets (LogNormal(0,1) scores, capped water-filling, cap 1)"
                            if w.head_budgets else "")
-                        + SELECTOR_TEXT[w.selector].format(seed=w.seed, stride=w.stride)
+                        + SELECTOR_TEXT[w.selector].format(seed=w.seed, stride=w.stride, rounds=w.rounds)
                         + (", special tokens read as patch tokens (no dense special path)"
                            if w.sparse_specials else "")
                         + KIND_TEXT[w.kind].format(T=w.tokens_per_frame, C=w.heads * w.head_dim),

@@ -152,6 +152,32 @@ BSA_API bsa_status bsa_probe_mask(const bsa_layout* layout, const float* pq, con
                                   const double* head_density, uint32_t* mask_bits, uint16_t* kv_idx,
                                   int32_t* kv_cnt, int32_t* status_dev, bsa_stream_t stream);
 
+/* Drift-score selection -- "ReSS: Residual-Restoring Sparse Attention for 3D Vision
+ * Transformers" (摘要, 技术框架, 关键设计: blocks chosen by the drift their removal leaves in the
+ * residual stream, refined by iterative residual restoration), read at the pooled resolution of
+ * bsa_predict_mask. Per head h and query block i, in fp64 from the fp32 pooled means:
+ *   p_j = softmax_j(pq[h,i] . pk[h,:,j] / sqrt(d)), o = sum_j p_j pv[h,:,j],
+ *   delta_j = p_j (o - pv[h,:,j]),
+ *   drift(D) = |sum_{j in D} delta_j| / (1 - sum_{j in D} p_j) for a dropped set D (the exact
+ *   shift of the renormalised pooled output).
+ * Keep the k_h blocks of largest |delta_j| (ties to the lower index); then, at most `rounds`
+ * times, restore the dropped block with the smallest resulting drift and drop the kept block
+ * (other than it) with the smallest resulting drift, keeping the swap only if the drift fell.
+ *   pq, pk : device, float32 [H, B, d] and [H, d, B] (bsa_pool_qk)
+ *   pv     : device, float32 [H, d, B] (bsa_pool_v)
+ *   rounds : 0 .. BSA_RESS_MAX_ROUNDS
+ * Needs P_b(V) of one head in shared memory: BSA_ERR_UNSUPPORTED above about B = 850 blocks. */
+#define BSA_RESS_MAX_ROUNDS 1024
+BSA_API bsa_status bsa_ress_mask(const bsa_layout* layout, const float* pq, const float* pk, const float* pv,
+                                 double rho, const double* head_density, int32_t rounds, uint32_t* mask_bits,
+                                 uint16_t* kv_idx, int32_t* kv_cnt, int32_t* status_dev, bsa_stream_t stream);
+
+/* Block pooling of V for bsa_ress_mask: pv[h, :, j] = the mean of V over the patch tokens of
+ * block j, fp32, dimension-major [H, d, B] (as pk).
+ *   v  : device, [N, H, d] of layout->dtype;  pv : device, float32 [H, d, B] */
+BSA_API bsa_status bsa_pool_v(const bsa_layout* layout, const void* v, float* pv, int32_t* status_dev,
+                              bsa_stream_t stream);
+
 /* ---------------------------------------------------------------------------------
  * Packing (prepares steps 4 and 5 for bf16 layers; the token split of 关键设计 3 made
  * physical). Copies the patch tokens and the special tokens of Q, K and V into a

@@ -46,8 +46,19 @@ def drift(delta: np.ndarray, p_row: np.ndarray, dropped: np.ndarray) -> float:
     return float(np.linalg.norm(delta[dropped].sum(axis=0))) / (1.0 - mass)
 
 
-def select_row(p_row: np.ndarray, pv: np.ndarray, k: int, rounds: int):
-    """Kept-block mask [B] of one row and the number of swaps taken."""
+def _gap(vals) -> float:
+    """Relative gap between the smallest and the second-smallest value (inf if fewer than 2)."""
+    v = np.sort(np.asarray(vals, dtype=np.float64))
+    if len(v) < 2 or not np.isfinite(v[1]):
+        return float("inf")
+    return float((v[1] - v[0]) / max(abs(v[0]), abs(v[1]), 1e-300))
+
+
+def select_row(p_row: np.ndarray, pv: np.ndarray, k: int, rounds: int, margins: list | None = None):
+    """Kept-block mask [B] of one row and the number of swaps taken. When `margins` is a list,
+    the relative gap of every decision is appended to it (the start cut, each argmin, each
+    keep-or-undo comparison), so that a comparison with another evaluation can tell a
+    rounding-level tie from a real difference."""
     B = len(p_row)
     k = min(max(k, 0), B)
     _, delta = drift_vectors(p_row, pv)
@@ -55,6 +66,8 @@ def select_row(p_row: np.ndarray, pv: np.ndarray, k: int, rounds: int):
     order = np.lexsort((np.arange(B), -norm))           # |delta| descending, index ascending
     kept = np.zeros(B, dtype=bool)
     kept[order[:k]] = True
+    if margins is not None and 0 < k < B:
+        margins.append(_gap([-norm[order[k - 1]], -norm[order[k]]]))
     if k == 0 or k == B:
         return kept, 0
     swaps = 0
@@ -63,13 +76,19 @@ def select_row(p_row: np.ndarray, pv: np.ndarray, k: int, rounds: int):
         # restore the dropped block whose return lowers the drift most
         cand = np.nonzero(~kept)[0]
         vals = [drift(delta, p_row, (~kept) & (np.arange(B) != l)) for l in cand]
+        if margins is not None:
+            margins.append(_gap(vals))
         l = int(cand[int(np.argmin(vals))])
         kept[l] = True
         # drop the kept block whose removal raises it least
         cand = np.nonzero(kept & (np.arange(B) != l))[0]
         vals = [drift(delta, p_row, (~kept) | (np.arange(B) == m)) for m in cand]
+        if margins is not None:
+            margins.append(_gap(vals))
         m = int(cand[int(np.argmin(vals))])
         new = min(vals)
+        if margins is not None:
+            margins.append(_gap([new, cur]))
         if new < cur:
             kept[m] = False
             swaps += 1

@@ -92,4 +92,30 @@ def test_no_writes_outside_the_buffers(w):
         a = g["out"].raw[g["out"].off: g["out"].off + n * 2].view(torch.bfloat16).float()
         b = g["out2"].raw[g["out2"].off: g["out2"].off + n * 2].view(torch.bfloat16).float()
         assert torch.linalg.vector_norm(a - b) <= 3e-3 * torch.linalg.vector_norm(a)
+    # the other block selectors write the same list buffers
+    run("random", lambda: _lib.bsa_random_mask(lay, w.rho, None, 7, P["mask_bits"], P["kv_idx"], P["kv_cnt"], sp, st))
+    run("uniform", lambda: _lib.bsa_uniform_mask(lay, 3, P["mask_bits"], P["kv_idx"], P["kv_cnt"], sp, st))
+    run("probe", lambda: _lib.bsa_probe_mask(lay, P["pq"], P["pk"], w.rho, None, P["mask_bits"], P["kv_idx"],
+                                             P["kv_cnt"], sp, st))
+    g["pv"] = Guarded(torch, H * d * B * 4)
+    P["pv"] = g["pv"].ptr
+    run("pool_v", lambda: _lib.bsa_pool_v(lay, vp, P["pv"], sp, st))
+    run("ress", lambda: _lib.bsa_ress_mask(lay, P["pq"], P["pk"], P["pv"], w.rho, None, 4, P["mask_bits"],
+                                           P["kv_idx"], P["kv_cnt"], sp, st))
+    if w.dtype == "bf16":
+        # the steps on either side of the layer
+        C = H * d
+        bi = synth.make_block_inputs(w)
+        xd, wq, wo = (layer.to_device(a, "bf16") for a in (bi.x, bi.w_qkv, bi.w_o))
+        bq, bo = torch.from_numpy(bi.b_qkv).cuda(), torch.from_numpy(bi.b_o).cuda()
+        for name in ("q2", "k2", "v2", "y"):
+            g[name] = Guarded(torch, N * C * 2)
+        fws = _lib.bsa_frame_workspace_size(lay)
+        g["fws"] = Guarded(torch, fws, align=1024)
+        P.update({n: g[n].ptr for n in ("q2", "k2", "v2", "y", "fws")})
+        run("qkv_project", lambda: _lib.bsa_qkv_project(lay, xd.data_ptr(), wq.data_ptr(), bq.data_ptr(), P["q2"],
+                                                        P["k2"], P["v2"], sp, st))
+        run("out_project", lambda: _lib.bsa_out_project(lay, P["q2"], wo.data_ptr(), bo.data_ptr(), P["y"], sp, st))
+        run("pack_frames", lambda: _lib.bsa_pack_frames(lay, qp, kp, vp, P["fws"], fws, sp, st))
+        run("frame_attention", lambda: _lib.bsa_frame_attention(lay, P["fws"], fws, P["out2"], sp, st))
     assert _lib.bsa_check_status(sp, st) == _lib.BSA_OK

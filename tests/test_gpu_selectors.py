@@ -172,3 +172,54 @@ def test_ablation_masks_and_layer(w):
     assert rep.ok, rep.failures
     _check_lists(sel, cnt, idx)
     _check_output(w, x, lay, sel, out)
+
+
+RESS = [
+    configs.RESS100.with_(name="ress_f3", **SMALL),
+    configs.RESS100.with_(name="ress_f3_b64", block=64, **SMALL),
+    configs.RESS100.with_(name="ress_f3_r0", rounds=0, **SMALL),
+    configs.RESS100.with_(name="ress_f4_rho_r32", frames=4, heads=3, head_budgets=False, rho=0.5, rounds=32),
+    configs.RESS100.with_(name="ress_f3_k0", head_budgets=False, rho=1.0, **SMALL),
+    configs.RESS100,
+]
+
+
+@pytest.mark.parametrize("w", RESS, ids=lambda w: w.name)
+def test_drift_score_selection(w):
+    """Drift-score rows ("ReSS...", 技术框架 / 关键设计) against the oracle run on the device's own
+    pooled means (fp32 values, exact in fp64), so that both sides take every decision in fp64
+    on the same numbers: rows must match exactly unless one of the oracle's decisions had a
+    relative gap below 1e-9 (a rounding-level tie). The pooled V is checked against the
+    oracle's pooling, and the layer output against the oracle fed the device's lists."""
+    from oracle import ress
+    x = inputs(w)
+    dens = head_density(w, x)
+    L, status, out, sel, cnt, idx = _run(w, x, dens)
+    assert status == 0
+    lay = _lay(w)
+    PQd = L.buf.pq.cpu().numpy().astype(np.float64)
+    PKd = L.buf.pk.cpu().numpy().astype(np.float64).transpose(0, 2, 1)
+    PVd = L.pv.cpu().numpy().astype(np.float64).transpose(0, 2, 1)
+    V = exact(x.v, w.dtype)
+    assert max_abs(PVd, oracle.pool(V, lay)) < 1e-5
+    kh = oracle.head_k(lay, w.rho, dens)
+    probs = oracle.pooled_probs(PQd, PKd, lay.head_dim)
+    H, B = lay.heads, lay.B
+    pairs = [(h, i) for h in range(H) for i in range(B)]
+    if len(pairs) > 400:
+        g = np.random.default_rng(11)
+        pairs = [pairs[t] for t in g.choice(len(pairs), 96, replace=False)]
+    exact_rows = exempt = 0
+    for h, i in pairs:
+        margins = []
+        ref, _ = ress.select_row(probs[h, i], PVd[h], int(kh[h]), w.rounds, margins)
+        if np.array_equal(ref, sel[h, i]):
+            exact_rows += 1
+        else:
+            assert margins and min(margins) < 1e-9, (h, i, np.nonzero(ref ^ sel[h, i])[0])
+            exempt += 1
+    print(f"{w.name}: rows {len(pairs)} exact {exact_rows} exempt {exempt}; density {sel.mean():.3f}")
+    assert np.array_equal(cnt, np.broadcast_to(np.minimum(kh, B)[:, None], cnt.shape))
+    _check_lists(sel, cnt, idx)
+    if np.any(kh > 0):
+        _check_output(w, x, lay, sel, out)

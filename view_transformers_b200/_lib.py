@@ -49,6 +49,9 @@ _SIGS = {
     "bsa_pack_frames": [_LP, _vp, _vp, _vp, _vp, _sz, _i32p, _st],
     "bsa_frame_attention": [_LP, _vp, _sz, _vp, _i32p, _st],
     "bsa_frame_workspace_size": [_LP, ctypes.POINTER(ctypes.c_size_t)],
+    "bsa_pool_v": [_LP, _vp, _vp, _i32p, _st],
+    "bsa_ress_mask": [_LP, _vp, _vp, _vp, ctypes.c_double, ctypes.c_void_p, ctypes.c_int32, _vp, _vp, _vp, _i32p,
+                      _st],
     "bsa_random_mask": [_LP, ctypes.c_double, ctypes.c_void_p, ctypes.c_uint64, _vp, _vp, _vp, _i32p, _st],
     "bsa_uniform_mask": [_LP, ctypes.c_int32, _vp, _vp, _vp, _i32p, _st],
     "bsa_probe_mask": [_LP, _vp, _vp, ctypes.c_double, ctypes.c_void_p, _vp, _vp, _vp, _i32p, _st],
@@ -176,6 +179,17 @@ def bsa_random_mask(layout, rho, head_density, seed, mask_bits, kv_idx, kv_cnt, 
     keep, dens = _densities(head_density)
     _check("bsa_random_mask", load().bsa_random_mask(ctypes.byref(layout), rho, dens, int(seed), mask_bits,
                                                      kv_idx, kv_cnt, status, stream))
+
+
+def bsa_pool_v(layout, v, pv, status=0, stream=0) -> None:
+    _check("bsa_pool_v", load().bsa_pool_v(ctypes.byref(layout), v, pv, status, stream))
+
+
+def bsa_ress_mask(layout, pq, pk, pv, rho, head_density, rounds, mask_bits, kv_idx, kv_cnt, status=0,
+                  stream=0) -> None:
+    keep, dens = _densities(head_density)
+    _check("bsa_ress_mask", load().bsa_ress_mask(ctypes.byref(layout), pq, pk, pv, rho, dens, int(rounds), mask_bits,
+                                                 kv_idx, kv_cnt, status, stream))
 
 
 def bsa_uniform_mask(layout, stride, mask_bits, kv_idx, kv_cnt, status=0, stream=0) -> None:

@@ -31,9 +31,11 @@ class Workload:
     head_budgets: bool = False  # per-head densities from capped water-filling
     seed: int = 0
     # block selector: "predict" (pooled softmax + dual threshold), "random" (k_h uniformly
-    # random blocks), "uniform" (every `stride`-th block), "probe" (mean-query Top-K)
+    # random blocks), "uniform" (every `stride`-th block), "probe" (mean-query Top-K), "ress"
+    # (drift scores with restoration rounds)
     selector: str = "predict"
     stride: int = 4
+    rounds: int = 8   # restoration rounds of the drift-score selector
     # the ablation without the dense special path: the layer reads the S special tokens of
     # every frame as patch tokens (pooled and sparsified with them)
     sparse_specials: bool = False
@@ -108,6 +110,9 @@ RANDOM_NOSPECIAL100 = PERHEAD100.with_(name="random_nospecial100", selector="ran
 # query-probe Top-K (the per-head budgets of the 100-frame workload).
 UNIFORM100 = PERHEAD100.with_(name="uniform100", selector="uniform", stride=4, head_budgets=False)
 PROBE100 = PERHEAD100.with_(name="probe100", selector="probe")
+# Drift-score selection of "ReSS: Residual-Restoring Sparse Attention for 3D Vision Transformers"
+# (技术框架 / 关键设计), with the per-head budgets of the 100-frame workload.
+RESS100 = PERHEAD100.with_(name="ress100", selector="ress")
 
 # The steps on either side of the layer ("Block-Sparse Global Attention...", 研究背景: the
 # aggregator alternates frame-wise and global attention; "SAF3R...", 图2): frame-wise dense
@@ -119,4 +124,4 @@ FRAME_BLOCK100 = PERHEAD100.with_(name="frame_block100", kind="frame_block", hea
 
 ALL = {w.name: w for w in (FRAME100, BLOCK100, FRAME_BLOCK100, TINY, VGGT518, SWEEP_R50, SWEEP_R75, SWEEP_R90, PERHEAD100,
                            PERHEAD100_TAU95, LONG500, TINY_TAU0, SWEEP_TAU0, CDF_ONLY100, NOSPECIAL100,
-                           RANDOM100, RANDOM_NOSPECIAL100, UNIFORM100, PROBE100)}
+                           RANDOM100, RANDOM_NOSPECIAL100, UNIFORM100, PROBE100, RESS100)}

@@ -41,6 +41,11 @@ cudaError_t launch_gemm_bf16(int M, int N, int K, const void* a, const void* b, 
 cudaError_t launch_pack_frames(const Geo& g, const void* q, const void* k, const void* v, void* ws,
                                int32_t* status, cudaStream_t st);
 cudaError_t launch_attn_frame(const Geo& g, const void* ws, void* out, int32_t* status, cudaStream_t st);
+cudaError_t launch_pool_v(const Geo& g, bsa_dtype dt, const void* v, float* pv, cudaStream_t st);
+size_t ress_smem_bytes(int B, int warps);
+cudaError_t launch_ress_mask(const Geo& g, const int* k_per_head, int rounds, const float* pq, const float* pk,
+                             const float* pv, uint32_t* mask_bits, uint16_t* kv_idx, int32_t* kv_cnt,
+                             cudaStream_t st);
 
 namespace {
 
@@ -404,6 +409,32 @@ bsa_status bsa_block_sparse_attn_fused(const bsa_layout* layout, const void* q, 
     if (s != BSA_OK) return s;
     return from_cuda(launch_attn_tc(g, 3, workspace, kv_idx, kv_cnt, nullptr, nullptr, out, status_dev,
                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
+bsa_status bsa_pool_v(const bsa_layout* layout, const void* v, float* pv, int32_t* status_dev, bsa_stream_t stream) {
+    (void)status_dev;
+    Geo g;
+    bsa_status s = make_geo(layout, &g);
+    if (s != BSA_OK) return s;
+    if (!v || !pv || !aligned16(v) || !aligned16(pv)) return BSA_ERR_INVALID_ARG;
+    return from_cuda(launch_pool_v(g, layout->dtype, v, pv, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+bsa_status bsa_ress_mask(const bsa_layout* layout, const float* pq, const float* pk, const float* pv, double rho,
+                         const double* head_density, int32_t rounds, uint32_t* mask_bits, uint16_t* kv_idx,
+                         int32_t* kv_cnt, int32_t* status_dev, bsa_stream_t stream) {
+    (void)status_dev;
+    Geo g;
+    bsa_status s = make_geo(layout, &g);
+    if (s != BSA_OK) return s;
+    if (!pq || !pk || !pv || !aligned16(pq) || !aligned16(pk) || !aligned16(pv) || !lists_ok(kv_idx, kv_cnt, mask_bits))
+        return BSA_ERR_INVALID_ARG;
+    if (rounds < 0 || rounds > BSA_RESS_MAX_ROUNDS) return BSA_ERR_INVALID_ARG;
+    if (ress_smem_bytes(g.B, 1) > 227u * 1024u) return BSA_ERR_UNSUPPORTED;
+    int k[BSA_MAX_HEADS];
+    if ((s = head_budgets_k(g, rho, head_density, k)) != BSA_OK) return s;
+    return from_cuda(launch_ress_mask(g, k, rounds, pq, pk, pv, mask_bits, kv_idx, kv_cnt,
+                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 
 bsa_status bsa_qkv_project(const bsa_layout* layout, const void* x, const void* w_qkv, const float* b_qkv,

@@ -17,15 +17,19 @@ namespace {
 constexpr int kPoolThreads = 256;
 constexpr int kChunksPerCta = 32;   // 16-byte chunks of a row per CTA (4 heads in bf16)
 
+// Tensor t = blockIdx.y + y0: t = 0 pools q into pq ([H][B][d]); t = 1 pools k into pk,
+// dimension-major ([H][d][B]).
 template <typename T>
 __global__ void __launch_bounds__(kPoolThreads)
 pool_kernel(Geo g, const T* __restrict__ q, const T* __restrict__ k, float* __restrict__ pq,
-            float* __restrict__ pk) {
+            float* __restrict__ pk, int y0) {
     extern __shared__ float red[];  // [ngroups][per_round * V] partial sums
     constexpr int V = Vec16<T>::n;
     const int j = blockIdx.x;
-    const T* src = blockIdx.y == 0 ? q : k;
-    float* dst = blockIdx.y == 0 ? pq : pk;
+    const int t = blockIdx.y + y0;
+    const T* src = t == 0 ? q : k;
+    float* dst = t == 0 ? pq : pk;
+    const bool dim_major = t == 1;
     const int row_elems = g.H * g.d;
     const int chunks = row_elems / V;                     // 16-byte chunks per row
     const int cbeg = blockIdx.z * kChunksPerCta;          // this CTA's chunks of every row
@@ -73,8 +77,8 @@ pool_kernel(Geo g, const T* __restrict__ q, const T* __restrict__ k, float* __re
             const int el = c0 * V + e;
             const int h = el / g.d;
             const int dd = el - h * g.d;
-            const size_t at = blockIdx.y == 0 ? ((size_t)h * g.B + j) * g.d + dd     // pq [H][B][d]
-                                              : ((size_t)h * g.d + dd) * g.B + j;    // pk [H][d][B]
+            const size_t at = !dim_major ? ((size_t)h * g.B + j) * g.d + dd     // [H][B][d]
+                                         : ((size_t)h * g.d + dd) * g.B + j;    // [H][d][B]
             dst[at] = s / count;
         }
         __syncthreads();
@@ -83,20 +87,34 @@ pool_kernel(Geo g, const T* __restrict__ q, const T* __restrict__ k, float* __re
 
 }  // namespace
 
-cudaError_t launch_pool(const Geo& g, bsa_dtype dt, const void* q, const void* k, float* pq,
-                        float* pk, cudaStream_t st) {
+namespace {
+// Tensors y0 .. y0 + tensors - 1 (0: q -> pq, 1: k -> pk dimension-major).
+cudaError_t launch_pool_tensors(const Geo& g, bsa_dtype dt, int y0, int tensors, const void* q, const void* k,
+                                float* pq, float* pk, cudaStream_t st) {
     const int V = dt == BSA_BF16 ? 8 : 4;
     const int chunks = g.H * g.d / V;
     const size_t smem = (size_t)kPoolThreads * V * sizeof(float);   // ngroups x per_round <= 256 chunks
-    const dim3 grid(g.B, 2, (chunks + kChunksPerCta - 1) / kChunksPerCta);
+    const dim3 grid(g.B, tensors, (chunks + kChunksPerCta - 1) / kChunksPerCta);
     if (dt == BSA_BF16) {
         pool_kernel<__nv_bfloat16><<<grid, kPoolThreads, smem, st>>>(
-            g, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), pq, pk);
+            g, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), pq, pk, y0);
     } else {
         pool_kernel<float><<<grid, kPoolThreads, smem, st>>>(
-            g, static_cast<const float*>(q), static_cast<const float*>(k), pq, pk);
+            g, static_cast<const float*>(q), static_cast<const float*>(k), pq, pk, y0);
     }
     return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_pool(const Geo& g, bsa_dtype dt, const void* q, const void* k, float* pq,
+                        float* pk, cudaStream_t st) {
+    return launch_pool_tensors(g, dt, 0, 2, q, k, pq, pk, st);
+}
+
+// P_b(V), dimension-major [H][d][B] (the layout the drift-score kernel stages in shared memory):
+// the K branch of the same kernel, run on V alone.
+cudaError_t launch_pool_v(const Geo& g, bsa_dtype dt, const void* v, float* pv, cudaStream_t st) {
+    return launch_pool_tensors(g, dt, 1, 1, nullptr, v, nullptr, pv, st);
 }
 
 }  // namespace bsa

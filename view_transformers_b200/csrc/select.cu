@@ -20,6 +20,7 @@
 // significant first, a 256-bin histogram in shared memory per pass) and then emits in
 // ascending index order with ballots. Integer work: results are exact.
 #include "common.cuh"
+#include "select.cuh"
 
 namespace bsa {
 namespace {
@@ -47,97 +48,12 @@ __device__ __forceinline__ uint32_t philox_word0(uint32_t c0, uint32_t c1, uint3
     return c0;
 }
 
-__device__ __forceinline__ unsigned lanemask_lt() {
-    unsigned m;
-    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
-    return m;
-}
-
 // Order-preserving 32-bit image of a float, reversed so that the largest score gets the
 // smallest key; -0 and +0 share one key.
 __device__ __forceinline__ uint32_t descending_key(float s) {
     const uint32_t u = __float_as_uint(s + 0.0f);
     const uint32_t up = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
     return ~up;
-}
-
-// One warp: of keys[0, n) (shared memory), keep the `need` entries with the smallest
-// (key, index). Writes the kept indices in ascending order to out[0, count) and, when
-// `bits` is not null, the row's kept-block bits (word w = blocks 32w .. 32w+31). `hist` is
-// 256 words of shared memory owned by the warp. Returns the count (min(need, n)).
-__device__ int warp_select_smallest(const uint32_t* keys, int n, int need, uint16_t* out, uint32_t* bits,
-                                    unsigned* hist) {
-    const int lane = threadIdx.x & 31;
-    uint32_t thr = 0u;
-    int take_eq = 0;   // entries equal to thr that are kept, lowest indices first
-    const bool all = need >= n;
-    if (!all && need > 0) {
-        uint32_t prefix = 0u, pmask = 0u;
-        int rem = need;
-        for (int shift = 24; shift >= 0; shift -= 8) {
-            for (int b = lane; b < 256; b += 32) hist[b] = 0u;
-            __syncwarp();
-            for (int j = lane; j < n; j += 32) {
-                const uint32_t u = keys[j];
-                if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1u);
-            }
-            __syncwarp();
-            // lane l owns digits 8l .. 8l+7; the digit where the running count reaches rem
-            unsigned c[8], local = 0u;
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                c[q] = hist[8 * lane + q];
-                local += c[q];
-            }
-            unsigned incl = local;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const unsigned v = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += v;
-            }
-            const unsigned excl = incl - local;
-            const unsigned hit = __ballot_sync(0xffffffffu, excl < (unsigned)rem && (unsigned)rem <= incl);
-            const int src = __ffs(hit) - 1;   // rem <= number of candidates, so one lane hits
-            int digit = 0;
-            unsigned before = 0u;
-            if (lane == src) {
-                unsigned acc = excl;
-                int q = 0;
-                while (q < 7 && acc + c[q] < (unsigned)rem) acc += c[q++];
-                digit = 8 * lane + q;
-                before = acc;
-            }
-            digit = __shfl_sync(0xffffffffu, digit, src);
-            before = __shfl_sync(0xffffffffu, before, src);
-            rem -= (int)before;
-            prefix |= (uint32_t)digit << shift;
-            pmask |= 0xffu << shift;
-            __syncwarp();
-        }
-        thr = prefix;
-        take_eq = rem;
-    }
-    int pos = 0, eq_seen = 0;
-    const unsigned lt_mask = lanemask_lt();
-    for (int base = 0; base < n; base += 32) {
-        const int j = base + lane;
-        const bool valid = j < n;
-        const uint32_t u = valid ? keys[j] : 0xffffffffu;
-        bool sel;
-        if (all) {
-            sel = valid;
-        } else {
-            const unsigned eqm = __ballot_sync(0xffffffffu, valid && u == thr && need > 0);
-            const int r = eq_seen + __popc(eqm & lt_mask);
-            sel = need > 0 && valid && (u < thr || (u == thr && r < take_eq));
-            eq_seen += __popc(eqm);
-        }
-        const unsigned sm = __ballot_sync(0xffffffffu, sel);
-        if (sel) out[pos + __popc(sm & lt_mask)] = (uint16_t)j;
-        pos += __popc(sm);
-        if (bits != nullptr && lane == 0) bits[base >> 5] = sm;
-    }
-    return pos;
 }
 
 struct SelParams {

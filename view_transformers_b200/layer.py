@@ -36,20 +36,21 @@ class Buffers:
 class BlockSparseLayer:
     """One global-attention layer of fixed geometry and selection hyper-parameters."""
 
-    SELECTORS = ("predict", "random", "uniform", "probe")
+    SELECTORS = ("predict", "random", "uniform", "probe", "ress")
 
     def __init__(self, frames: int, tokens_per_frame: int, special_per_frame: int, heads: int,
                  head_dim: int, block: int, dtype: str, rho: float, tau: float, head_density=None,
                  device: str | torch.device = "cuda", selector: str = "predict", seed: int = 0,
-                 stride: int = 4):
+                 stride: int = 4, rounds: int = 8):
         """selector: how the kept blocks are chosen -- "predict" (pooled softmax and the dual
         threshold), "random" (k_h blocks uniformly at random, keyed by `seed`), "uniform"
-        (every `stride`-th block) or "probe" (the k_h blocks of highest mean-query score)."""
+        (every `stride`-th block), "probe" (the k_h blocks of highest mean-query score) or
+        "ress" (the k_h blocks by drift score, refined by up to `rounds` restoration swaps)."""
         if selector not in self.SELECTORS:
             raise ValueError(f"selector must be one of {self.SELECTORS}")
         self.layout = _lib.make_layout(frames, tokens_per_frame, special_per_frame, heads, head_dim, block, dtype)
         self.dtype = dtype
-        self.selector, self.seed, self.stride = selector, int(seed), int(stride)
+        self.selector, self.seed, self.stride, self.rounds = selector, int(seed), int(stride), int(rounds)
         self.rho, self.tau = float(rho), float(tau)
         self.head_density = None if head_density is None else [float(x) for x in head_density]
         self.device = torch.device(device)
@@ -70,28 +71,38 @@ class BlockSparseLayer:
             out=torch.empty((self.N, H, d), dtype=_TORCH_DTYPE[dtype], device=dev),
             status=torch.zeros(1, dtype=torch.int32, device=dev),
         )
+        # pooled V, dimension-major [H, d, B], for the drift-score selector
+        self.pv = torch.empty((H, d, B), dtype=torch.float32, device=dev) if selector == "ress" else None
         base = self.buf.workspace.data_ptr()
         self.ws_ptr = (base + 1023) // 1024 * 1024 if self.ws_bytes else 0
 
     @classmethod
     def for_workload(cls, w, head_density=None, device="cuda") -> "BlockSparseLayer":
         return cls(w.frames, w.tokens_per_frame, w.layer_special, w.heads, w.head_dim, w.block,
-                   w.dtype, w.rho, w.tau, head_density, device, w.selector, w.seed, w.stride)
+                   w.dtype, w.rho, w.tau, head_density, device, w.selector, w.seed, w.stride, w.rounds)
 
     # individual steps -------------------------------------------------------------
-    def predict(self, q: torch.Tensor, k: torch.Tensor, stream: int | None = None) -> None:
+    def predict(self, q: torch.Tensor, k: torch.Tensor, stream: int | None = None, v: torch.Tensor | None = None) -> None:
+        """Block selection from Q and K (and V for the drift-score selector)."""
         st = self._stream(stream)
         b = self.buf
-        if self.selector in ("predict", "probe"):
+        if self.selector in ("predict", "probe", "ress"):
             _lib.bsa_pool_qk(self.layout, q.data_ptr(), k.data_ptr(), b.pq.data_ptr(), b.pk.data_ptr(),
                              b.status.data_ptr(), st)
-        self._select(st)
+        self._select(st, v)
 
-    def _select(self, st) -> None:
-        """The block selection step, from the pooled means already in pq / pk."""
+    def _select(self, st, v: torch.Tensor | None = None) -> None:
+        """The block selection step, from the pooled means already in pq / pk (the drift-score
+        selector also pools v)."""
         b = self.buf
         args = (b.mask_bits.data_ptr(), b.kv_idx.data_ptr(), b.kv_cnt.data_ptr(), b.status.data_ptr(), st)
-        if self.selector == "predict":
+        if self.selector == "ress":
+            if v is None:
+                raise ValueError("the drift-score selector needs v")
+            _lib.bsa_pool_v(self.layout, v.data_ptr(), self.pv.data_ptr(), b.status.data_ptr(), st)
+            _lib.bsa_ress_mask(self.layout, b.pq.data_ptr(), b.pk.data_ptr(), self.pv.data_ptr(), self.rho,
+                               self.head_density, self.rounds, *args)
+        elif self.selector == "predict":
             _lib.bsa_predict_mask(self.layout, b.pq.data_ptr(), b.pk.data_ptr(), self.rho, self.tau,
                                   self.head_density, *args)
         elif self.selector == "random":
@@ -153,7 +164,7 @@ class BlockSparseLayer:
         if fused is None:
             fused = self.dtype == "bf16"
         if not fused:
-            self.predict(q, k, stream)
+            self.predict(q, k, stream, v)
             return self.attend(q, k, v, stream, out)
         st = self._stream(stream)
         b = self.buf
@@ -162,12 +173,12 @@ class BlockSparseLayer:
         # packing and pooling in one pass over Q, K, V; then mask, special rows, patch rows.
         # (Running the special rows on a second stream next to the mask and the patch rows
         # was measured slower: both attention passes are compute-bound and share the SMs.)
-        if self.selector in ("predict", "probe"):
+        if self.selector in ("predict", "probe", "ress"):
             _lib.bsa_pack_pool_qkv(self.layout, qp, kp, vp, self.ws_ptr, self.ws_bytes, b.pq.data_ptr(),
                                    b.pk.data_ptr(), b.status.data_ptr(), st)
         else:   # the selection reads no pooled means
             _lib.bsa_pack_qkv(self.layout, qp, kp, vp, self.ws_ptr, self.ws_bytes, b.status.data_ptr(), st)
-        self._select(st)
+        self._select(st, v)
         _lib.bsa_special_dense(self.layout, qp, kp, vp, self.ws_ptr, self.ws_bytes, o.data_ptr(),
                                None, None, b.status.data_ptr(), st)
         main = None
