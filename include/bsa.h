@@ -164,13 +164,18 @@ BSA_API bsa_status bsa_probe_mask(const bsa_layout* layout, const float* pq, con
  * times, restore the dropped block with the smallest resulting drift and drop the kept block
  * (other than it) with the smallest resulting drift, keeping the swap only if the drift fell.
  *   pq, pk : device, float32 [H, B, d] and [H, d, B] (bsa_pool_qk)
- *   pv     : device, float32 [H, d, B] (bsa_pool_v)
- *   rounds : 0 .. BSA_RESS_MAX_ROUNDS
- * Needs P_b(V) of one head in shared memory: BSA_ERR_UNSUPPORTED above about B = 850 blocks. */
+ *   pv        : device, float32 [H, d, B] (bsa_pool_v)
+ *   rounds    : 0 .. BSA_RESS_MAX_ROUNDS
+ *   workspace : device, 16-byte aligned, at least bsa_ress_workspace_size() bytes (the fp64
+ *               Gram matrix of pv per head, H B B doubles; overwritten)
+ * Needs P_b(V) of one head in shared memory: BSA_ERR_UNSUPPORTED above about B = 800 blocks. */
 #define BSA_RESS_MAX_ROUNDS 1024
 BSA_API bsa_status bsa_ress_mask(const bsa_layout* layout, const float* pq, const float* pk, const float* pv,
-                                 double rho, const double* head_density, int32_t rounds, uint32_t* mask_bits,
-                                 uint16_t* kv_idx, int32_t* kv_cnt, int32_t* status_dev, bsa_stream_t stream);
+                                 double rho, const double* head_density, int32_t rounds, void* workspace,
+                                 size_t workspace_bytes, uint32_t* mask_bits, uint16_t* kv_idx, int32_t* kv_cnt,
+                                 int32_t* status_dev, bsa_stream_t stream);
+/* Bytes of bsa_ress_mask's workspace: H B B 8. */
+BSA_API bsa_status bsa_ress_workspace_size(const bsa_layout* layout, size_t* bytes);
 
 /* Block pooling of V for bsa_ress_mask: pv[h, :, j] = the mean of V over the patch tokens of
  * block j, fp32, dimension-major [H, d, B] (as pk).

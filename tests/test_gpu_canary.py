@@ -100,8 +100,11 @@ def test_no_writes_outside_the_buffers(w):
     g["pv"] = Guarded(torch, H * d * B * 4)
     P["pv"] = g["pv"].ptr
     run("pool_v", lambda: _lib.bsa_pool_v(lay, vp, P["pv"], sp, st))
-    run("ress", lambda: _lib.bsa_ress_mask(lay, P["pq"], P["pk"], P["pv"], w.rho, None, 4, P["mask_bits"],
-                                           P["kv_idx"], P["kv_cnt"], sp, st))
+    rws = _lib.bsa_ress_workspace_size(lay)
+    g["rws"] = Guarded(torch, rws)
+    P["rws"] = g["rws"].ptr
+    run("ress", lambda: _lib.bsa_ress_mask(lay, P["pq"], P["pk"], P["pv"], w.rho, None, 4, P["rws"], rws,
+                                           P["mask_bits"], P["kv_idx"], P["kv_cnt"], sp, st))
     if w.dtype == "bf16":
         # the steps on either side of the layer
         C = H * d

@@ -50,8 +50,9 @@ _SIGS = {
     "bsa_frame_attention": [_LP, _vp, _sz, _vp, _i32p, _st],
     "bsa_frame_workspace_size": [_LP, ctypes.POINTER(ctypes.c_size_t)],
     "bsa_pool_v": [_LP, _vp, _vp, _i32p, _st],
-    "bsa_ress_mask": [_LP, _vp, _vp, _vp, ctypes.c_double, ctypes.c_void_p, ctypes.c_int32, _vp, _vp, _vp, _i32p,
-                      _st],
+    "bsa_ress_mask": [_LP, _vp, _vp, _vp, ctypes.c_double, ctypes.c_void_p, ctypes.c_int32, _vp, _sz, _vp, _vp,
+                      _vp, _i32p, _st],
+    "bsa_ress_workspace_size": [_LP, ctypes.POINTER(ctypes.c_size_t)],
     "bsa_random_mask": [_LP, ctypes.c_double, ctypes.c_void_p, ctypes.c_uint64, _vp, _vp, _vp, _i32p, _st],
     "bsa_uniform_mask": [_LP, ctypes.c_int32, _vp, _vp, _vp, _i32p, _st],
     "bsa_probe_mask": [_LP, _vp, _vp, ctypes.c_double, ctypes.c_void_p, _vp, _vp, _vp, _i32p, _st],
@@ -185,11 +186,17 @@ def bsa_pool_v(layout, v, pv, status=0, stream=0) -> None:
     _check("bsa_pool_v", load().bsa_pool_v(ctypes.byref(layout), v, pv, status, stream))
 
 
-def bsa_ress_mask(layout, pq, pk, pv, rho, head_density, rounds, mask_bits, kv_idx, kv_cnt, status=0,
-                  stream=0) -> None:
+def bsa_ress_workspace_size(layout) -> int:
+    out = ctypes.c_size_t()
+    _check("bsa_ress_workspace_size", load().bsa_ress_workspace_size(ctypes.byref(layout), ctypes.byref(out)))
+    return out.value
+
+
+def bsa_ress_mask(layout, pq, pk, pv, rho, head_density, rounds, workspace, workspace_bytes, mask_bits, kv_idx,
+                  kv_cnt, status=0, stream=0) -> None:
     keep, dens = _densities(head_density)
-    _check("bsa_ress_mask", load().bsa_ress_mask(ctypes.byref(layout), pq, pk, pv, rho, dens, int(rounds), mask_bits,
-                                                 kv_idx, kv_cnt, status, stream))
+    _check("bsa_ress_mask", load().bsa_ress_mask(ctypes.byref(layout), pq, pk, pv, rho, dens, int(rounds), workspace,
+                                                 workspace_bytes, mask_bits, kv_idx, kv_cnt, status, stream))
 
 
 def bsa_uniform_mask(layout, stride, mask_bits, kv_idx, kv_cnt, status=0, stream=0) -> None:

@@ -43,9 +43,10 @@ cudaError_t launch_pack_frames(const Geo& g, const void* q, const void* k, const
 cudaError_t launch_attn_frame(const Geo& g, const void* ws, void* out, int32_t* status, cudaStream_t st);
 cudaError_t launch_pool_v(const Geo& g, bsa_dtype dt, const void* v, float* pv, cudaStream_t st);
 size_t ress_smem_bytes(int B, int warps);
+size_t ress_workspace_bytes(const Geo& g);
 cudaError_t launch_ress_mask(const Geo& g, const int* k_per_head, int rounds, const float* pq, const float* pk,
-                             const float* pv, uint32_t* mask_bits, uint16_t* kv_idx, int32_t* kv_cnt,
-                             cudaStream_t st);
+                             const float* pv, void* workspace, uint32_t* mask_bits, uint16_t* kv_idx,
+                             int32_t* kv_cnt, cudaStream_t st);
 
 namespace {
 
@@ -420,9 +421,19 @@ bsa_status bsa_pool_v(const bsa_layout* layout, const void* v, float* pv, int32_
     return from_cuda(launch_pool_v(g, layout->dtype, v, pv, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+bsa_status bsa_ress_workspace_size(const bsa_layout* layout, size_t* bytes) {
+    if (bytes == nullptr) return BSA_ERR_INVALID_ARG;
+    Geo g;
+    const bsa_status s = make_geo(layout, &g);
+    if (s != BSA_OK) return s;
+    *bytes = ress_workspace_bytes(g);
+    return BSA_OK;
+}
+
 bsa_status bsa_ress_mask(const bsa_layout* layout, const float* pq, const float* pk, const float* pv, double rho,
-                         const double* head_density, int32_t rounds, uint32_t* mask_bits, uint16_t* kv_idx,
-                         int32_t* kv_cnt, int32_t* status_dev, bsa_stream_t stream) {
+                         const double* head_density, int32_t rounds, void* workspace, size_t workspace_bytes,
+                         uint32_t* mask_bits, uint16_t* kv_idx, int32_t* kv_cnt, int32_t* status_dev,
+                         bsa_stream_t stream) {
     (void)status_dev;
     Geo g;
     bsa_status s = make_geo(layout, &g);
@@ -430,10 +441,12 @@ bsa_status bsa_ress_mask(const bsa_layout* layout, const float* pq, const float*
     if (!pq || !pk || !pv || !aligned16(pq) || !aligned16(pk) || !aligned16(pv) || !lists_ok(kv_idx, kv_cnt, mask_bits))
         return BSA_ERR_INVALID_ARG;
     if (rounds < 0 || rounds > BSA_RESS_MAX_ROUNDS) return BSA_ERR_INVALID_ARG;
+    if (workspace == nullptr || !aligned16(workspace) || workspace_bytes < ress_workspace_bytes(g))
+        return BSA_ERR_INVALID_ARG;
     if (ress_smem_bytes(g.B, 1) > 227u * 1024u) return BSA_ERR_UNSUPPORTED;
     int k[BSA_MAX_HEADS];
     if ((s = head_budgets_k(g, rho, head_density, k)) != BSA_OK) return s;
-    return from_cuda(launch_ress_mask(g, k, rounds, pq, pk, pv, mask_bits, kv_idx, kv_cnt,
+    return from_cuda(launch_ress_mask(g, k, rounds, pq, pk, pv, workspace, mask_bits, kv_idx, kv_cnt,
                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 

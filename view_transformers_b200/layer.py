@@ -71,8 +71,10 @@ class BlockSparseLayer:
             out=torch.empty((self.N, H, d), dtype=_TORCH_DTYPE[dtype], device=dev),
             status=torch.zeros(1, dtype=torch.int32, device=dev),
         )
-        # pooled V, dimension-major [H, d, B], for the drift-score selector
+        # pooled V, dimension-major [H, d, B], and the Gram-matrix workspace of the drift-score selector
         self.pv = torch.empty((H, d, B), dtype=torch.float32, device=dev) if selector == "ress" else None
+        self.ress_ws_bytes = _lib.bsa_ress_workspace_size(self.layout) if selector == "ress" else 0
+        self.ress_ws = torch.empty(max(self.ress_ws_bytes, 1), dtype=torch.uint8, device=dev) if selector == "ress" else None
         base = self.buf.workspace.data_ptr()
         self.ws_ptr = (base + 1023) // 1024 * 1024 if self.ws_bytes else 0
 
@@ -101,7 +103,7 @@ class BlockSparseLayer:
                 raise ValueError("the drift-score selector needs v")
             _lib.bsa_pool_v(self.layout, v.data_ptr(), self.pv.data_ptr(), b.status.data_ptr(), st)
             _lib.bsa_ress_mask(self.layout, b.pq.data_ptr(), b.pk.data_ptr(), self.pv.data_ptr(), self.rho,
-                               self.head_density, self.rounds, *args)
+                               self.head_density, self.rounds, self.ress_ws.data_ptr(), self.ress_ws_bytes, *args)
         elif self.selector == "predict":
             _lib.bsa_predict_mask(self.layout, b.pq.data_ptr(), b.pk.data_ptr(), self.rho, self.tau,
                                   self.head_density, *args)
