@@ -8,9 +8,6 @@
 //                      partials in the workspace, combined by special_combine_kernel
 //   MODE_FUSED         patch query tile over the special keys and the kept key blocks in
 //                      one online softmax: steps 4, 5(ii) and the merge in one pass -> out
-//   MODE_FRAME         query tile of one frame over every key of the same frame (the frame-
-//                      wise attention that alternates with the global one, 研究背景), from the
-//                      per-frame packing of pack.cu -> out
 //
 // Inputs come from the packed workspace (pack.cu): per head, 64-wide rows of 128 bytes,
 // so a query tile (128 rows) is one 2D TMA box with the 128-byte swizzle that the MMA
@@ -69,7 +66,7 @@ constexpr float kRescale = 8.0f;                     // lazy-rescale threshold (
 constexpr float kLn2 = 0.69314718055994531f;
 constexpr int kThreads = 192;
 
-enum { MODE_SPARSE = 0, MODE_PATCH_SPECIAL = 1, MODE_SPECIAL_ALL = 2, MODE_FUSED = 3, MODE_FRAME = 4 };
+enum { MODE_SPARSE = 0, MODE_PATCH_SPECIAL = 1, MODE_SPECIAL_ALL = 2, MODE_FUSED = 3 };
 
 struct TcParams {
     Geo g;
@@ -83,7 +80,6 @@ struct TcParams {
     float* slse;
     int32_t* status;
     int q_tiles;   // query tiles per head
-    int frame_pad;   // MODE_FRAME: packed rows per (head, frame), a multiple of 128
 };
 
 // BKV is the block size b (64 or 128). Query and key tiles are always 128 rows: a key tile
@@ -150,12 +146,6 @@ struct TileWalk {
     __device__ __forceinline__ bool next(int u, const Geo& g, const PackedLayout& pl, int h, int sp_tiles,
                                          int t_begin, Tile& t) {
         t.member = (1u << (KB * QB)) - 1u;
-        if (MODE == MODE_FRAME) {   // t_begin: first packed row of the frame
-            t.special = false;
-            t.row0[0] = t_begin + u * 128;
-            t.nvalid[0] = min(128, g.T - u * 128);
-            return true;
-        }
         if (MODE == MODE_SPECIAL_ALL) {
             const int x = t_begin + u;
             t.special = x < sp_tiles;
@@ -262,11 +252,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     const int sp_tiles = (g.Ns + 127) / 128;       // special key tiles (128 rows)
     int t_begin = 0, t_end = 0;                    // MODE_SPECIAL_ALL key-tile range
-    // MODE_FRAME: frame of the query tile, its tile within the frame and the frame's key tiles
-    const int f_tiles = MODE == MODE_FRAME ? prm.frame_pad / 128 : 1;
-    const int frame = MODE == MODE_FRAME ? tq / f_tiles : 0;
-    const int ftile = MODE == MODE_FRAME ? tq - frame * f_tiles : 0;
-    if (MODE == MODE_FRAME) t_begin = (h * g.F + frame) * prm.frame_pad;
     if (MODE == MODE_SPECIAL_ALL) {
         const int n_all = sp_tiles + pl.np_pad / 128;   // even split: sizes differ by at most one
         t_begin = (int)((long long)split * n_all / pl.nsplit);
@@ -354,16 +339,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int n = MODE == MODE_SPARSE ? kept_tiles
                 : MODE == MODE_FUSED ? sp_tiles + kept_tiles
                 : MODE == MODE_PATCH_SPECIAL ? sp_tiles
-                : MODE == MODE_FRAME ? f_tiles
                 : t_end - t_begin;
     int issued = 0;   // K/V tiles whose loads the producer issued
 
     if (warp == 0) {
         // ============================================================ TMA producer
         if (lane == 0) {
-            const int q_row0 = MODE == MODE_SPECIAL_ALL ? h * pl.ns_pad + tq * 128
-                             : MODE == MODE_FRAME ? t_begin + ftile * 128
-                             : h * pl.np_pad + tq * 128;
+            const int q_row0 = MODE == MODE_SPECIAL_ALL ? h * pl.ns_pad + tq * 128 : h * pl.np_pad + tq * 128;
             mbar_arrive_expect_tx(&ctl.q_full, 128 * 128);
             tma_load_2d(smem + C::kOffQ, &tm_q, &ctl.q_full, 0, q_row0);
             TileWalk<MODE, BKV> walk(bits, words);
@@ -639,13 +621,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 float* dst = prm.spart + (((size_t)split * g.H + h) * pl.ns_pad + qrow) * 64 + 32 * a;
 #pragma unroll
                 for (int c = 0; c < 32; c += 4) Vec16<float>::store(dst + c, o + c);
-            } else if (MODE == MODE_FRAME) {
-                const int r = ftile * 128 + row;
-                if (r < g.T) {
-                    __nv_bfloat16* dst = prm.out + ((size_t)frame * g.T + r) * g.H * 64 + (size_t)h * 64 + 32 * a;
-#pragma unroll
-                    for (int c = 0; c < 32; c += 8) Vec16<__nv_bfloat16>::store(dst + c, o + c);
-                }
             } else if (MODE == MODE_FUSED) {
                 if (qrow < g.Np) {
                     __nv_bfloat16* dst = prm.out + (size_t)patch_row(g, qrow) * g.H * 64 + (size_t)h * 64 + 32 * a;
@@ -659,7 +634,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
         }
         if (MODE == MODE_SPECIAL_ALL) prm.slse[((size_t)split * g.H + h) * pl.ns_pad + qrow] = lse;
-        else if (MODE != MODE_FUSED && MODE != MODE_FRAME && qrow < g.Np) prm.lse_part[(size_t)h * g.Np + qrow] = lse;
+        else if (MODE != MODE_FUSED && qrow < g.Np) prm.lse_part[(size_t)h * g.Np + qrow] = lse;
     }
 
     // ------------------------------------------------------------------ teardown
@@ -757,26 +732,6 @@ cudaError_t launch_mode(const TcParams& prm, const CUtensorMap& q, const CUtenso
 }
 
 }  // namespace
-
-// Frame-wise attention: every query tile of a frame over the key tiles of the same frame, from
-// the per-frame packing (frame_layout) in ws; writes every row of out (bf16).
-cudaError_t launch_attn_frame(const Geo& g, const void* ws, void* out, int32_t* status, cudaStream_t st) {
-    const FrameLayout fl = frame_layout(g);
-    uint8_t* base = static_cast<uint8_t*>(const_cast<void*>(ws));
-    TcParams prm{};
-    prm.g = g;
-    prm.pl = packed_layout(g);
-    prm.out = static_cast<__nv_bfloat16*>(out);
-    prm.status = status;
-    prm.frame_pad = fl.t_pad;
-    prm.q_tiles = g.F * (fl.t_pad / 128);
-    const uint64_t rows = (uint64_t)g.H * g.F * fl.t_pad;
-    CUtensorMap q, k, v;
-    if (!make_map(&q, base + fl.qf, rows, 128, false) || !make_map(&k, base + fl.kf, rows, 128, false) ||
-        !make_map(&v, base + fl.vf, rows, 128, true))
-        return cudaErrorInvalidValue;
-    return launch_mode<MODE_FRAME, 128>(prm, q, k, v, k, v, prm.q_tiles * g.H, st);
-}
 
 // mode: 0 sparse (o_part/lse_part), 1 patch->special (o_part/lse_part),
 //       2 special->all (out, through the split partials), 3 fused sparse + special keys (out)
