@@ -165,3 +165,49 @@ def test_head_budgets_validation(lib):
     assert lib.bsa_head_budgets(s, 3, 0.5, 1.0, d) == E.BSA_ERR_INVALID_ARG
     s2 = (ctypes.c_double * 3)(1.0, 1.0, 2.0)
     assert lib.bsa_head_budgets(s2, 3, 0.5, 0.1, d) == E.BSA_ERR_INVALID_ARG   # budget above H * cap
+
+
+def test_selector_and_projection_argument_validation(lib):
+    """The selectors, the projections and the frame-wise attention reject bad arguments on the
+    host, before anything is launched (A is never dereferenced)."""
+    lay = ctypes.byref(_lay())
+    # random selection: rho in [0, 1], lists required and aligned; densities validated as in the mask
+    assert lib.bsa_random_mask(lay, 1.5, None, 0, None, A, A, None, None) == E.BSA_ERR_INVALID_ARG
+    assert lib.bsa_random_mask(lay, 0.5, None, 0, None, None, A, None, None) == E.BSA_ERR_INVALID_ARG
+    assert lib.bsa_random_mask(lay, 0.5, None, 0, A + 4, A, A, None, None) == E.BSA_ERR_INVALID_ARG
+    dens = (ctypes.c_double * 2)(0.5, 0.6)
+    assert lib.bsa_random_mask(lay, 0.5, dens, 0, None, A, A, None, None) == E.BSA_ERR_INVALID_ARG
+    # uniform sampling: stride >= 1
+    assert lib.bsa_uniform_mask(lay, 0, None, A, A, None, None) == E.BSA_ERR_INVALID_ARG
+    assert lib.bsa_uniform_mask(lay, 2, None, A, None, None, None) == E.BSA_ERR_INVALID_ARG
+    # query probe: pooled tensors required
+    assert lib.bsa_probe_mask(lay, None, A, 0.5, None, None, A, A, None, None) == E.BSA_ERR_INVALID_ARG
+    assert lib.bsa_probe_mask(lay, A, A, -0.1, None, None, A, A, None, None) == E.BSA_ERR_INVALID_ARG
+    # drift scores: rounds in range, workspace large enough, pooled V required
+    rws = ctypes.c_size_t()
+    assert lib.bsa_ress_workspace_size(lay, ctypes.byref(rws)) == E.BSA_OK
+    assert rws.value == 2 * 8 * 8 * 8                                    # H B B doubles, B = 8
+    assert lib.bsa_ress_mask(lay, A, A, A, 0.5, None, -1, A, rws.value, None, A, A, None, None) == E.BSA_ERR_INVALID_ARG
+    assert lib.bsa_ress_mask(lay, A, A, A, 0.5, None, 2000, A, rws.value, None, A, A, None,
+                             None) == E.BSA_ERR_INVALID_ARG
+    assert lib.bsa_ress_mask(lay, A, A, A, 0.5, None, 4, A, rws.value - 1, None, A, A, None,
+                             None) == E.BSA_ERR_INVALID_ARG
+    assert lib.bsa_ress_mask(lay, A, A, None, 0.5, None, 4, A, rws.value, None, A, A, None,
+                             None) == E.BSA_ERR_INVALID_ARG
+    big = _lay(frames=100, tokens_per_frame=782, block=64, dtype="bf16")   # B = 1215: P_b(V) exceeds shared memory
+    assert lib.bsa_ress_mask(ctypes.byref(big), A, A, A, 0.5, None, 4, A, 1 << 40, None, A, A, None,
+                             None) == E.BSA_ERR_UNSUPPORTED
+    assert lib.bsa_pool_v(lay, None, A, None, None) == E.BSA_ERR_INVALID_ARG
+    # projections and frame-wise attention: bf16 layouts only, pointers required
+    assert lib.bsa_qkv_project(lay, A, A, None, A, A, A, None, None) == E.BSA_ERR_UNSUPPORTED          # f32 layout
+    bf = ctypes.byref(_lay(dtype="bf16", block=64))
+    assert lib.bsa_qkv_project(bf, A, A, None, A, None, A, None, None) == E.BSA_ERR_INVALID_ARG
+    assert lib.bsa_qkv_project(bf, A, A, A + 4, A, A, A, None, None) == E.BSA_ERR_INVALID_ARG        # bias misaligned
+    assert lib.bsa_out_project(bf, A, None, None, A, None, None) == E.BSA_ERR_INVALID_ARG
+    fws = ctypes.c_size_t()
+    assert lib.bsa_frame_workspace_size(bf, ctypes.byref(fws)) == E.BSA_OK
+    assert fws.value == 3 * 2 * 2 * 128 * 128                            # H F t_pad rows of 128 bytes, x3
+    assert lib.bsa_pack_frames(bf, A, A, A, A, fws.value - 1, None, None) == E.BSA_ERR_INVALID_ARG
+    assert lib.bsa_pack_frames(bf, A, A, A, A + 16, fws.value, None, None) == E.BSA_ERR_INVALID_ARG  # 1024-byte alignment
+    assert lib.bsa_frame_attention(bf, A, fws.value, None, None, None) == E.BSA_ERR_INVALID_ARG
+    assert lib.bsa_frame_attention(lay, A, fws.value, A, None, None) == E.BSA_ERR_UNSUPPORTED          # f32 layout
