@@ -21,6 +21,9 @@
 //   o_final             committed after the item's last P.V; the softmax waits on it, reads O,
 //                       writes the rows, and only then arrives on p_full of the next item's
 //                       first tile, so the next item's first P.V (which overwrites O) follows.
+// A frame's last key tile holds T mod 128 keys (14 at T = 782): its QK^T runs at N = the keys
+// rounded up to 16, its P.V over the 16-key steps that hold keys, and the softmax skips the
+// exponentials and P stores of the 32-key chunks past T.
 // Every wait is bounded; a timeout is reported through the status word.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -139,14 +142,17 @@ frame_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     } else if (warp == 1) {
         // ============================================================ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc_qk = idesc_f16(128, 128, 1u, false);
             constexpr uint32_t idesc_pv = idesc_f16(128, 64, 0u, true);
             const uint32_t q_base = smem_u32(smem + kFOffQ);
-            auto issue_qk = [&](int U) -> bool {
+            // QK^T of key tile u of an item, over its keys rounded up to 16 (a frame's last
+            // tile holds T mod 128 keys)
+            auto issue_qk = [&](int U, int u) -> bool {
                 const int st = U % kFStages;
                 if (!mbar_wait(&ctl.kv_full[st], (U / kFStages) & 1, abort, prm.status)) return false;
                 tc_fence_after();
                 const uint32_t k_base = smem_u32(smem + kFOffK + st * kFTile);
+                const int n16 = (min(128, g.T - u * 128) + 15) & ~15;
+                const uint32_t idesc_qk = idesc_f16(128, n16, 1u, false);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
                     mma_ss(tmem + kFColS, sdesc_sw128(q_base + 32 * ks, 16, 1024), sdesc_sw128(k_base + 32 * ks, 16, 1024),
@@ -160,23 +166,25 @@ frame_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (!mbar_wait(&ctl.q_full, I & 1, abort, prm.status)) break;
                 // the previous item's last S has been read by the softmax
                 if (I > 0 && !mbar_wait(&ctl.s_free, (U - 1) & 1, abort, prm.status)) break;
-                if (!(ok = issue_qk(U))) break;
+                if (!(ok = issue_qk(U, 0))) break;
                 if (nt == 1) mma_commit(&ctl.q_empty);
                 for (int u = 0; u < nt; ++u) {
                     const int Uu = U + u;
                     if (u + 1 < nt) {
                         if (!mbar_wait(&ctl.s_free, Uu & 1, abort, prm.status)) { ok = false; break; }
-                        if (!(ok = issue_qk(Uu + 1))) break;
+                        if (!(ok = issue_qk(Uu + 1, u + 1))) break;
                         if (u + 2 == nt) mma_commit(&ctl.q_empty);   // the item's last QK^T is issued
                     }
                     if (!mbar_wait(&ctl.p_full, Uu & 1, abort, prm.status)) { ok = false; break; }
                     tc_fence_after();
                     const int st = Uu % kFStages;
                     const uint32_t v_base = smem_u32(smem + kFOffV + st * kFTile);
+                    const int k16 = (min(128, g.T - u * 128) + 15) / 16;   // 16-key steps holding keys
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks)
-                        mma_ts(tmem + kFColO, tmem + kFColP + 8 * ks, sdesc_sw128(v_base + 2048 * ks, 0, 1024), idesc_pv,
-                               (u > 0 || ks > 0) ? 1u : 0u);
+                        if (ks < k16)
+                            mma_ts(tmem + kFColO, tmem + kFColP + 8 * ks, sdesc_sw128(v_base + 2048 * ks, 0, 1024),
+                                   idesc_pv, (u > 0 || ks > 0) ? 1u : 0u);
                     mma_commit(&ctl.kv_empty[st]);
                     mma_commit(&ctl.o_done);
                     if (u == nt - 1) mma_commit(&ctl.o_final);
@@ -247,13 +255,24 @@ frame_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     }
                     rs = ((r2[0].x + r2[0].y) + (r2[1].x + r2[1].y)) + ((r2[2].x + r2[2].y) + (r2[3].x + r2[3].y));
                 } else {
+                    // the frame's last tile: chunks of 32 keys, those past T skipped (warp-uniform)
 #pragma unroll
-                    for (int c = 0; c < 128; c += 2) {
-                        const float p0 = c < nvalid ? ex2_approx(fmaf(__uint_as_float(s[c]), kFScaleLog2, -m_ref)) : 0.f;
-                        const float p1 =
-                            c + 1 < nvalid ? ex2_approx(fmaf(__uint_as_float(s[c + 1]), kFScaleLog2, -m_ref)) : 0.f;
-                        rs += p0 + p1;
-                        s[c / 2] = pack_half2(p0, p1);
+                    for (int k = 0; k < 4; ++k) {
+                        if (32 * k < nvalid) {
+#pragma unroll
+                            for (int c = 32 * k; c < 32 * k + 32; c += 2) {
+                                const float p0 =
+                                    c < nvalid ? ex2_approx(fmaf(__uint_as_float(s[c]), kFScaleLog2, -m_ref)) : 0.f;
+                                const float p1 =
+                                    c + 1 < nvalid ? ex2_approx(fmaf(__uint_as_float(s[c + 1]), kFScaleLog2, -m_ref))
+                                                   : 0.f;
+                                rs += p0 + p1;
+                                s[c / 2] = pack_half2(p0, p1);
+                            }
+                        } else {
+#pragma unroll
+                            for (int c = 32 * k; c < 32 * k + 32; c += 2) s[c / 2] = 0u;
+                        }
                     }
                 }
                 l = l * factor + rs;
@@ -273,8 +292,9 @@ frame_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     }
                 }
 #pragma unroll
-                for (int c = 0; c < 2; ++c)
-                    tmem_st32(lane_base + kFColP + 32 * c, *reinterpret_cast<const uint32_t(*)[32]>(&s[32 * c]));
+                for (int c = 0; c < 2; ++c)   // P.V reads only the 16-key steps that hold keys
+                    if (64 * c < nvalid)
+                        tmem_st32(lane_base + kFColP + 32 * c, *reinterpret_cast<const uint32_t(*)[32]>(&s[32 * c]));
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
