@@ -54,6 +54,8 @@ PROJ = [
     configs.VGGT518.with_(name="proj_h16", frames=3),               # C = 1024, N = 4122 (ragged M)
     configs.VGGT518.with_(name="proj_h2", frames=2, heads=2),       # C = 128: 3C = 384, partial N tile
     configs.VGGT518.with_(name="proj_h3", frames=1, heads=3),       # C = 192: 3C = 576, tiles straddle q/k
+    # fewer rows than one 256-row tile of a CTA pair: the second CTA's rows all lie past the end
+    configs.VGGT518.with_(name="proj_m105", frames=1, heads=2, patch_per_frame=100),
     configs.PERHEAD100,                                             # full size, sampled rows
 ]
 
