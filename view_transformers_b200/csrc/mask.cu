@@ -416,7 +416,9 @@ mask_kernel(Geo g, MaskParams mp, const float* __restrict__ pq, const float* __r
 
     // ---- pooled scores: work items of 32 blocks (one per lane) x RG rows, round-robin over
     // the warps (consecutive warps take consecutive block chunks)
-    constexpr int RG = R <= 9 ? R : 8;   // rows per work item; R is a multiple of RG
+    // rows per work item (R is a multiple of RG): every row at once, unless several CTAs
+    // share the SM and registers cap the accumulators at 9
+    constexpr int RG = (MINB == 1 || R <= 9) ? R : 8;
     const float* pk_h = pk + (size_t)h * kDim * B;
     const float scale = 0.125f;   // 1 / sqrt(64)
     const int nchunk = (B + 31) / 32;
@@ -508,7 +510,7 @@ cudaError_t launch_mask(const Geo& g, const MaskParams& mp, const float* pq, con
     // each other's barrier. When the rows leave a small last round of CTAs (e.g. 2.05 rounds
     // of 4 x 148 CTAs at 100 frames), 9 rows on 9 warps (at most 56 registers, so that four
     // CTAs still fit) finish in one round fewer.
-    // With long rows only one CTA fits on an SM: 16 warps then keep the score pass busier.
+    // With long rows only one CTA fits on an SM: as many rows as fit (one warp each).
     const size_t per_sm = 228 * 1024;
     const int slots = num_sms() * 4;
     const long long ctas8 = (long long)((g.B + 7) / 8) * g.H, ctas9 = (long long)((g.B + 8) / 9) * g.H;
@@ -519,6 +521,12 @@ cudaError_t launch_mask(const Geo& g, const MaskParams& mp, const float* pq, con
     const size_t limit = 227 * 1024;
     // (the launch bounds keep every variant within 64 registers per thread)
     if (small) return launch_rows<8, kWarps, 4>(g, mp, pq, pk, mask_bits, kv_idx, kv_cnt, status, st);
+    // Long rows: one CTA per SM, one warp per row in both phases (no warp idles during the
+    // selection), all rows of the CTA in each score work item (one pass over pooled K)
+    if (mask_smem<14>(g.B, 14) <= limit)
+        return launch_rows<14, 14, 1>(g, mp, pq, pk, mask_bits, kv_idx, kv_cnt, status, st);
+    if (mask_smem<12>(g.B, 12) <= limit)
+        return launch_rows<12, 12, 1>(g, mp, pq, pk, mask_bits, kv_idx, kv_cnt, status, st);
     if (mask_smem<8>(g.B, 2 * kWarps) <= limit)
         return launch_rows<8, 2 * kWarps, 2>(g, mp, pq, pk, mask_bits, kv_idx, kv_cnt, status, st);
     if (mask_smem<4>(g.B, 2 * kWarps) <= limit)
