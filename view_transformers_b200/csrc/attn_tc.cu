@@ -24,10 +24,10 @@
 //               p = 2^(s log2(e)/sqrt(d) - m) in fp32, P rounded to fp16 into TMEM,
 //               then the epilogue O / l and the log-sum-exp.
 // For b = 64 a 128-row query tile holds two query blocks; it walks the union of their
-// kept blocks, two per 128-key tile. The softmax computes every column of a tile whose kept
-// blocks are whole and then drops, by selects, the block a row's query block did not keep
-// (from the row max, the row sum and P); only tiles with a ragged kept block go column by
-// column.
+// kept blocks, two per 128-key tile. A warp's 32 rows share a query block, so the softmax
+// branches per warp on which of the tile's two key blocks that query block kept: both (all
+// 128 columns), one (its 64 columns, P = 0 for the other) or neither (P = 0); only tiles
+// with a ragged kept block go column by column.
 //
 // Barrier protocol (u = tile index of the CTA). A parity wait only tells apart phases
 // within one phase of the barrier's current one; every wait below has that property:
@@ -511,27 +511,55 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             float rs = 0.f;
             if constexpr (KB == 2) {
                 if (full) {
-                    // every column, then the halves this row's query block did not keep are
-                    // dropped from the sum and from P (their p may be inf: never used)
-                    float2 r2[4];   // [0, 1]: first half, [2, 3]: second half
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) r2[i] = make_float2(0.f, 0.f);
+                    // only the halves this row's query block kept (warp-uniform: a warp's 32
+                    // rows share a query block); a half it did not keep gives P = 0
                     const float2 scale2 = make_float2(kScaleLog2, kScaleLog2);
                     const float2 shift2 = make_float2(-m_ref, -m_ref);
+                    if (member && mem1) {
+                        float2 r2[4];
 #pragma unroll
-                    for (int c = 0; c < TC; c += 2) {
-                        const int i = c / 2;
-                        const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
-                                                    scale2, shift2);
-                        const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-                        r2[(c < 64 ? 0 : 2) + (i & 1)] = __fadd2_rn(r2[(c < 64 ? 0 : 2) + (i & 1)], pr);
-                        s[i] = pack_half2(pr.x, pr.y);
+                        for (int i = 0; i < 4; ++i) r2[i] = make_float2(0.f, 0.f);
+#pragma unroll
+                        for (int c = 0; c < TC; c += 2) {
+                            const int i = c / 2;
+                            const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
+                                                        scale2, shift2);
+                            const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                            r2[i & 3] = __fadd2_rn(r2[i & 3], pr);
+                            s[i] = pack_half2(pr.x, pr.y);
+                        }
+                        rs = ((r2[0].x + r2[0].y) + (r2[1].x + r2[1].y)) + ((r2[2].x + r2[2].y) + (r2[3].x + r2[3].y));
+                    } else if (member) {   // first half only
+                        float2 r2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+                        for (int c = 0; c < 64; c += 2) {
+                            const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
+                                                        scale2, shift2);
+                            const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                            r2[(c / 2) & 1] = __fadd2_rn(r2[(c / 2) & 1], pr);
+                            s[c / 2] = pack_half2(pr.x, pr.y);
+                        }
+#pragma unroll
+                        for (int i = 32; i < 64; ++i) s[i] = 0u;
+                        rs = (r2[0].x + r2[0].y) + (r2[1].x + r2[1].y);
+                    } else if (mem1) {     // second half only
+                        float2 r2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+                        for (int c = 64; c < 128; c += 2) {
+                            const float2 x = __ffma2_rn(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
+                                                        scale2, shift2);
+                            const float2 pr = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                            r2[(c / 2) & 1] = __fadd2_rn(r2[(c / 2) & 1], pr);
+                            s[c / 2] = pack_half2(pr.x, pr.y);
+                        }
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) s[i] = 0u;
+                        rs = (r2[0].x + r2[0].y) + (r2[1].x + r2[1].y);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 64; ++i) s[i] = 0u;
+                        rs = 0.f;
                     }
-                    const float r0 = (r2[0].x + r2[0].y) + (r2[1].x + r2[1].y);
-                    const float r1 = (r2[2].x + r2[2].y) + (r2[3].x + r2[3].y);
-                    rs = (member ? r0 : 0.f) + (mem1 ? r1 : 0.f);
-#pragma unroll
-                    for (int i = 0; i < 64; ++i) s[i] = (i < 32 ? member : mem1) ? s[i] : 0u;
                 } else {
 #pragma unroll
                     for (int c = 0; c < TC; c += 2) {
