@@ -287,9 +287,8 @@ BSA_API bsa_status bsa_block_sparse_attn_fused(const bsa_layout* layout, const v
 /* ---------------------------------------------------------------------------------
  * The steps on either side of the layer. The pages put the global attention inside an
  * aggregator that alternates frame-wise and global multi-head attention ("Block-Sparse Global
- * Attention for Efficient Multi-View Geometry Transformers", 研究背景: 交替「帧内注意力 + 全局
- * 注意力」; "SAF3R: Dynamic Sparse Attention for Feed-Forward 3D Reconstruction Transformers",
- * 图2). bf16 layouts only (BSA_ERR_UNSUPPORTED otherwise); fp32 accumulation, bf16 results
+ * Attention for Efficient Multi-View Geometry Transformers", 研究背景与动机; "SAF3R: Dynamic Sparse
+ * Attention for Feed-Forward 3D Reconstruction Transformers", 图2). bf16 layouts only (BSA_ERR_UNSUPPORTED otherwise); fp32 accumulation, bf16 results
  * rounded to nearest even. C = heads * head_dim channels.
  *
  * QKV projection: [q | k | v] = x W_qkv^T + b_qkv, channel c of each third = head c / d,
@@ -298,7 +297,7 @@ BSA_API bsa_status bsa_block_sparse_attn_fused(const bsa_layout* layout, const v
  *   w_qkv  : device, bf16 [3C, C] (output features x input features, row-major)
  *   b_qkv  : device, float32 [3C], or NULL for no bias
  *   q, k, v: device, bf16 [N, H, d] each
- * tcgen05 MMA (128 x 256 output tiles, TMEM accumulators, TMA operand tiles). */
+ * tcgen05 MMA on CTA pairs (256 x 256 output tiles, TMEM accumulators, TMA operand tiles). */
 BSA_API bsa_status bsa_qkv_project(const bsa_layout* layout, const void* x, const void* w_qkv, const float* b_qkv,
                                    void* q, void* k, void* v, int32_t* status_dev, bsa_stream_t stream);
 

@@ -4,10 +4,10 @@ import it, and it imports nothing from the CUDA package).
 
 The pages place the global attention inside an aggregator that alternates frame-wise and
 global attention blocks, each a multi-head self-attention with its projections
-("Block-Sparse Global Attention for Efficient Multi-View Geometry Transformers", 研究背景 /
-领域现状: 交替「帧内注意力 + 全局注意力」; "SAF3R: Dynamic Sparse Attention for Feed-Forward 3D
-Reconstruction Transformers", 图2: alternating local and global attention modules of MHA and
-FFN). These are the steps written here:
+("Block-Sparse Global Attention for Efficient Multi-View Geometry Transformers", 研究背景与动机:
+the VGGT aggregator; "SAF3R: Dynamic Sparse Attention for Feed-Forward 3D Reconstruction
+Transformers", 图2: local and global attention modules, each multi-head attention plus a
+feed-forward network). These are the steps written here:
 
   * linear        y = x W^T + b (the QKV and output projections);
   * qkv_project   the QKV projection of C = H d channels into 3C, split as [Q | K | V], each

@@ -114,7 +114,7 @@ PROBE100 = PERHEAD100.with_(name="probe100", selector="probe")
 # (技术框架 / 关键设计), with the per-head budgets of the 100-frame workload.
 RESS100 = PERHEAD100.with_(name="ress100", selector="ress")
 
-# The steps on either side of the layer ("Block-Sparse Global Attention...", 研究背景: the
+# The steps on either side of the layer ("Block-Sparse Global Attention...", 研究背景与动机: the
 # aggregator alternates frame-wise and global attention; "SAF3R...", 图2): frame-wise dense
 # attention over the 782 tokens of each frame as a second workload, and whole blocks with the
 # QKV and output projections (random-init weights).

@@ -1,6 +1,6 @@
 // Frame-wise dense attention on the tensor cores: every token attends over the T tokens of its
 // own frame (the frame half of the aggregator that alternates frame-wise and global attention,
-// "Block-Sparse Global Attention for Efficient Multi-View Geometry Transformers", 研究背景;
+// "Block-Sparse Global Attention for Efficient Multi-View Geometry Transformers", 研究背景与动机;
 // "SAF3R: Dynamic Sparse Attention for Feed-Forward 3D Reconstruction Transformers", 图2).
 //
 // Input: the per-frame packing of pack.cu (frame_layout): per head and frame, the frame's T

@@ -1,7 +1,7 @@
 // Projections on either side of the attention layer: y = x W^T + b with bf16 inputs, fp32
 // accumulation and bf16 outputs. The pages place the global attention between the QKV and
 // output projections of a multi-head attention block ("Block-Sparse Global Attention for
-// Efficient Multi-View Geometry Transformers", 研究背景: the alternating frame / global
+// Efficient Multi-View Geometry Transformers", 研究背景与动机: the alternating frame / global
 // attention aggregator; "SAF3R: Dynamic Sparse Attention for Feed-Forward 3D Reconstruction
 // Transformers", 图2).
 //
