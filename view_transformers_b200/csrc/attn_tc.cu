@@ -43,14 +43,13 @@
 //   o_final  single phase, committed after the last P.V: the epilogue waits on it.
 // Every wait is bounded; a timeout is reported through the status word.
 #include <cuda.h>
-#include <cudaTypedefs.h>
 
 #include <cmath>
-#include <mutex>
 
 #include "common.cuh"
 #include "sm100.cuh"
 #include "tc_layout.cuh"
+#include "tma_map.cuh"
 
 namespace bsa {
 namespace {
@@ -720,33 +719,6 @@ special_combine_kernel(Geo g, PackedLayout pl, const float* __restrict__ spart, 
 
 // ---------------------------------------------------------------------- host side
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
-// 2D map over `rows` rows of 64 two-byte elements (128-byte pitch), box of box_rows rows.
-bool make_map(CUtensorMap* tm, const void* base, uint64_t rows, uint32_t box_rows, bool fp16) {
-    auto enc = get_encode();
-    if (enc == nullptr || rows == 0) return false;
-    cuuint64_t dims[2] = {64, rows};
-    cuuint64_t strides[1] = {128};
-    cuuint32_t box[2] = {64, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return enc(tm, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-               const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int MODE, int BKV>
 cudaError_t launch_mode(const TcParams& prm, const CUtensorMap& q, const CUtensorMap& ka, const CUtensorMap& va,
                         const CUtensorMap& kb, const CUtensorMap& vb, int ctas, cudaStream_t st) {
@@ -785,11 +757,11 @@ cudaError_t launch_attn_tc(const Geo& g, int mode, const void* ws, const uint16_
     CUtensorMap q, ka, va, kb, vb;
     const int patch_tiles = pl.np_pad / 128;
     if (mode == MODE_SPARSE || mode == MODE_FUSED) {
-        if (!make_map(&q, base + pl.qp, prow, 128, false) || !make_map(&kb, base + pl.kp, prow, g.b, false) ||
-            !make_map(&vb, base + pl.vp, prow, g.b, true))
+        if (!make_tile_map(&q, base + pl.qp, prow, 64, 128, false) || !make_tile_map(&kb, base + pl.kp, prow, 64, g.b, false) ||
+            !make_tile_map(&vb, base + pl.vp, prow, 64, g.b, true))
             return cudaErrorInvalidValue;
         if (mode == MODE_FUSED && has_sp) {
-            if (!make_map(&ka, base + pl.ks, srow, g.b, false) || !make_map(&va, base + pl.vs, srow, g.b, true))
+            if (!make_tile_map(&ka, base + pl.ks, srow, 64, g.b, false) || !make_tile_map(&va, base + pl.vs, srow, 64, g.b, true))
                 return cudaErrorInvalidValue;
         } else {
             ka = kb;
@@ -804,15 +776,15 @@ cudaError_t launch_attn_tc(const Geo& g, int mode, const void* ws, const uint16_
                           : launch_mode<MODE_FUSED, 64>(prm, q, ka, va, kb, vb, ctas, st);
     }
     if (!has_sp) return cudaSuccess;
-    if (!make_map(&ka, base + pl.ks, srow, 128, false) || !make_map(&va, base + pl.vs, srow, 128, true))
+    if (!make_tile_map(&ka, base + pl.ks, srow, 64, 128, false) || !make_tile_map(&va, base + pl.vs, srow, 64, 128, true))
         return cudaErrorInvalidValue;
     if (mode == MODE_PATCH_SPECIAL) {
-        if (!make_map(&q, base + pl.qp, prow, 128, false)) return cudaErrorInvalidValue;
+        if (!make_tile_map(&q, base + pl.qp, prow, 64, 128, false)) return cudaErrorInvalidValue;
         prm.q_tiles = patch_tiles;
         return launch_mode<MODE_PATCH_SPECIAL, 128>(prm, q, ka, va, ka, va, patch_tiles * g.H, st);
     }
-    if (!make_map(&q, base + pl.qs, srow, 128, false) || !make_map(&kb, base + pl.kp, prow, 128, false) ||
-        !make_map(&vb, base + pl.vp, prow, 128, true))
+    if (!make_tile_map(&q, base + pl.qs, srow, 64, 128, false) || !make_tile_map(&kb, base + pl.kp, prow, 64, 128, false) ||
+        !make_tile_map(&vb, base + pl.vp, prow, 64, 128, true))
         return cudaErrorInvalidValue;
     prm.q_tiles = pl.ns_pad / 128;
     cudaError_t e = launch_mode<MODE_SPECIAL_ALL, 128>(prm, q, ka, va, kb, vb, prm.q_tiles * pl.nsplit * g.H, st);

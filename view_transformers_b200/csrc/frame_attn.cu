@@ -26,14 +26,13 @@
 // exponentials and P stores of the 32-key chunks past T.
 // Every wait is bounded; a timeout is reported through the status word.
 #include <cuda.h>
-#include <cudaTypedefs.h>
 
 #include <cmath>
-#include <mutex>
 
 #include "common.cuh"
 #include "sm100.cuh"
 #include "tc_layout.cuh"
+#include "tma_map.cuh"
 
 namespace bsa {
 namespace {
@@ -347,33 +346,6 @@ frame_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 frame_encode() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
-// 2D map over `rows` rows of 64 two-byte elements (128-byte pitch), 128-row boxes, 128-byte swizzle.
-bool frame_map(CUtensorMap* tm, const void* base, uint64_t rows, bool fp16) {
-    auto enc = frame_encode();
-    if (enc == nullptr || rows == 0) return false;
-    cuuint64_t dims[2] = {64, rows};
-    cuuint64_t strides[1] = {128};
-    cuuint32_t box[2] = {64, 128};
-    cuuint32_t estr[2] = {1, 1};
-    return enc(tm, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-               const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 }  // namespace
 
 // Frame-wise attention over the per-frame packing in ws; writes every row of out (bf16).
@@ -389,8 +361,8 @@ cudaError_t launch_attn_frame(const Geo& g, const void* ws, void* out, int32_t* 
     prm.status = status;
     const uint64_t rows = (uint64_t)g.H * g.F * fl.t_pad;
     CUtensorMap q, k, v;
-    if (!frame_map(&q, base + fl.qf, rows, false) || !frame_map(&k, base + fl.kf, rows, false) ||
-        !frame_map(&v, base + fl.vf, rows, true))
+    if (!make_tile_map(&q, base + fl.qf, rows, 64, 128, false) || !make_tile_map(&k, base + fl.kf, rows, 64, 128, false) ||
+        !make_tile_map(&v, base + fl.vf, rows, 64, 128, true))
         return cudaErrorInvalidValue;
     if (prm.items == 0) return cudaSuccess;
     const size_t smem = kFOffCtl + (sizeof(FCtl) + 15) / 16 * 16;

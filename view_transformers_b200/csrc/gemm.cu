@@ -26,6 +26,7 @@
 
 #include "common.cuh"
 #include "sm100.cuh"
+#include "tma_map.cuh"
 
 namespace bsa {
 namespace {
@@ -398,32 +399,6 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
     }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
-// Row-major [rows, cols] bf16 matrix, box of 64 columns x box_rows rows, 128-byte swizzle.
-bool make_kmajor_map(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-    auto enc = encode_fn();
-    if (enc == nullptr) return false;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {(cuuint32_t)kBK, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 constexpr size_t kPairSmem = kPStages * kPStageBytes + sizeof(PairCtl);
 
 // Clusters of two gemm_pair_kernel CTAs the current device holds at once (0: use the
@@ -458,7 +433,7 @@ cudaError_t launch_gemm_bf16(int M, int N, int K, const void* a, const void* b, 
     if (M <= 0 || N <= 0 || K <= 0 || K % kBK != 0 || N % 32 != 0 || split % 32 != 0 || N > 3 * split)
         return cudaErrorInvalidValue;
     CUtensorMap ta, tb;
-    if (!make_kmajor_map(&ta, a, (uint64_t)M, (uint64_t)K, kBM) || !make_kmajor_map(&tb, b, (uint64_t)N, (uint64_t)K, kBN))
+    if (!make_tile_map(&ta, a, (uint64_t)M, (uint64_t)K, kBM, false) || !make_tile_map(&tb, b, (uint64_t)N, (uint64_t)K, kBN, false))
         return cudaErrorInvalidValue;
     GemmParams prm;
     prm.M = M;
@@ -472,7 +447,7 @@ cudaError_t launch_gemm_bf16(int M, int N, int K, const void* a, const void* b, 
     const int pairs = pair_clusters();
     if (pairs > 0) {
         CUtensorMap tbp;
-        if (!make_kmajor_map(&tbp, b, (uint64_t)N, (uint64_t)K, 128)) return cudaErrorInvalidValue;
+        if (!make_tile_map(&tbp, b, (uint64_t)N, (uint64_t)K, 128, false)) return cudaErrorInvalidValue;
         const long long tiles = (long long)((M + 255) / 256) * ((N + 255) / 256);
         const int grid = 2 * (int)(tiles < pairs ? tiles : pairs);
         gemm_pair_kernel<<<grid, kGemmThreads, kPairSmem, st>>>(ta, tbp, prm);
