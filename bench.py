@@ -255,21 +255,43 @@ def run_steps(torch, L, q, k, v, steps, path="fused"):
 
 
 # ---------------------------------------------------------------------------- CPU oracle
-def oracle_layer_sample(w, x, budget_s: float, seed: int = 7):
+def oracle_layer_sample(w, x, budget_s: float, seed: int = 7, keep: dict | None = None):
     """Times the fp64 oracle on a bounded sample of one layer and scales it to ms/layer.
 
     Full pooling and mask prediction; attention for a seeded sample of (head, query block)
-    pairs plus a seeded sample of special query rows, scaled by the sampled fraction."""
+    pairs plus a seeded sample of special query rows, scaled by the sampled fraction. When
+    `keep` is a dict it receives the oracle's mask result and the outputs of the first
+    sampled pairs and special rows, for a parity check of the same run."""
     import oracle
     from threadpoolctl import threadpool_info, threadpool_limits
     host_cpus = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
     with threadpool_limits(limits=host_cpus):           # the BLAS pools use every host CPU
         threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-        est, sample = _oracle_layer_sample(oracle, w, x, budget_s, seed)
+        est, sample = _oracle_layer_sample(oracle, w, x, budget_s, seed, keep)
     return est, threads, host_cpus, sample
 
 
-def _oracle_layer_sample(oracle, w, x, budget_s, seed):
+def sample_parity(torch, L, w, keep: dict) -> dict:
+    """The benchmarked run's output and mask against the oracle on the CPU leg's sample:
+    relative L2 and max-abs over the kept rows (oracle run with its own mask), and the mask
+    of every row under the near-tie rule (the dual-threshold selector only)."""
+    from oracle.compare import compare_mask, max_abs, rel_l2
+    got, ref = [], []
+    out = L.buf.out
+    for rows, h, o in keep["rows"]:
+        idx = torch.as_tensor(rows, device=out.device)
+        got.append(out[idx, h].float().cpu().numpy())
+        ref.append(o)
+    got, ref = np.concatenate(got), np.concatenate(ref)
+    rep = {"rows": int(len(ref)), "rel_l2": rel_l2(got, ref), "max_abs": max_abs(got, ref),
+           "against": "the oracle's own mask, rows of the first sampled (head, query block) pairs and special rows"}
+    if keep.get("mask") is not None:
+        m = compare_mask(keep["mask"], L.selected(), w.tau)
+        rep["mask"] = {"rows": m.rows, "exact": m.exact, "near_tie_exempt": m.exempt, "failed": m.failed}
+    return rep
+
+
+def _oracle_layer_sample(oracle, w, x, budget_s, seed, keep=None):
     from oracle import selectors
     lay = oracle.Layout(w.frames, w.tokens_per_frame, w.layer_special, w.heads, w.head_dim, w.block)
     t0 = time.perf_counter()
@@ -277,7 +299,10 @@ def _oracle_layer_sample(oracle, w, x, budget_s, seed):
     dens = None if x.scores is None else oracle.water_fill(x.scores, w.heads * (1 - w.rho), 1.0)
     kh = oracle.head_k(lay, w.rho, dens)
     if w.selector == "predict":
-        selected = oracle.predict_mask(oracle.pool(Q, lay), oracle.pool(K, lay), lay.head_dim, kh, w.tau).selected
+        mres = oracle.predict_mask(oracle.pool(Q, lay), oracle.pool(K, lay), lay.head_dim, kh, w.tau)
+        selected = mres.selected
+        if keep is not None:
+            keep["mask"] = mres
     elif w.selector == "random":
         selected = selectors.random_mask(lay, kh, w.seed)
     elif w.selector == "uniform":
@@ -302,7 +327,9 @@ def _oracle_layer_sample(oracle, w, x, budget_s, seed):
         kept = selected[h, i] if selected is not None else ress.select_row(probs[h, i], PV[h], int(kh[h]),
                                                                           w.rounds)[0]
         keys = np.concatenate([sr, oracle.patch_keys_of(lay, kept)])
-        oracle.attend(Q[rows, h], K[keys, h], V[keys, h])
+        o = oracle.attend(Q[rows, h], K[keys, h], V[keys, h])[0]
+        if keep is not None and done < 16:
+            keep.setdefault("rows", []).append((rows, h, o))
         done += 1
         if time.perf_counter() - t1 > budget_s * 0.8:
             break
@@ -312,7 +339,9 @@ def _oracle_layer_sample(oracle, w, x, budget_s, seed):
     if lay.Ns:
         for h in range(lay.heads):
             rows = sr[g.choice(len(sr), size=min(8, len(sr)), replace=False)]
-            oracle.attend(Q[rows, h], K[:, h], V[:, h])
+            o = oracle.attend(Q[rows, h], K[:, h], V[:, h])[0]
+            if keep is not None:
+                keep.setdefault("rows", []).append((rows, h, o))
             n_spec_rows += len(rows)
     t_spec = time.perf_counter() - t2
     total_pairs = lay.heads * lay.B
@@ -781,7 +810,10 @@ def main():
         "clocks": clocks, "device_status": status,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        ms, threads, host_cpus, sample = oracle_layer_sample(w, x, budget_s=args.cpu_budget)
+        keep = {}
+        ms, threads, host_cpus, sample = oracle_layer_sample(w, x, budget_s=args.cpu_budget, keep=keep)
+        if keep.get("rows"):
+            line["parity_sample"] = sample_parity(torch, L, w, keep)
         line["cpu_baseline"] = {"value": ms, "unit": UNIT, "cores": threads, "host_cpus": host_cpus,
                                 "kind": "oracle", "extrapolated": True, "sample": sample}
     if rank == 0:
