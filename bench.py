@@ -283,7 +283,8 @@ def sample_parity(torch, L, w, keep: dict) -> dict:
         got.append(out[idx, h].float().cpu().numpy())
         ref.append(o)
     got, ref = np.concatenate(got), np.concatenate(ref)
-    rep = {"rows": int(len(ref)), "rel_l2": rel_l2(got, ref), "max_abs": max_abs(got, ref),
+    r = rel_l2(got, ref)
+    rep = {"rows": int(len(ref)), "rel_l2": r, "nmse": r * r, "max_abs": max_abs(got, ref),
            "against": "the oracle's own mask, rows of the first sampled (head, query block) pairs and special rows"}
     if keep.get("mask") is not None:
         m = compare_mask(keep["mask"], L.selected(), w.tau)
