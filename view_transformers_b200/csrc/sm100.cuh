@@ -1,6 +1,7 @@
 // Thin inline-PTX wrappers for the Blackwell (sm_100a) features used by the tensor-core
 // kernels: mbarriers with bounded waits, TMA tile loads, tcgen05 MMA / TMEM access.
-// Written from the PTX ISA; no multicast forms are used anywhere in this library.
+// Written from the PTX ISA. No TMA or bulk load in this library uses cluster multicast; the one
+// multicast form is a tcgen05.commit that arrives on both CTAs of a pair (no data moves).
 #pragma once
 
 #include <cstdint>
