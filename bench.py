@@ -533,6 +533,44 @@ def block_stage_calls(w, L, tensors, status, sp):
     return calls
 
 
+def block_parity_sample(torch, w, t, seed: int = 11) -> dict:
+    """The benchmarked frame-wise step against the oracle on sampled rows of two frames, each
+    stage on the device's own input to it: the QKV projection from x (block workloads), the
+    frame attention from the device's Q, K, V, the output projection from the device's
+    attention output. Relative L2 and max-abs per stage."""
+    from oracle import layer_io
+    from oracle.compare import max_abs, rel_l2
+    g = np.random.default_rng(seed)
+    T, H = w.tokens_per_frame, w.heads
+    frames = [int(f) for f in g.choice(w.frames, size=min(2, w.frames), replace=False)]
+    dev = t["o"].device
+    host = lambda a: a.float().cpu().numpy().astype(np.float64)
+    rep = {}
+
+    def stage(got, ref):
+        got, ref = np.concatenate(got), np.concatenate(ref)
+        return {"values": int(ref.size), "rel_l2": rel_l2(got, ref), "max_abs": max_abs(got, ref)}
+
+    if "y" in t:
+        rows = torch.as_tensor([f * T + int(r) for f in frames for r in g.integers(0, T, 16)], device=dev)
+        want = layer_io.qkv_project(host(t["x"][rows]), host(t["w_qkv"]), t["b_qkv"].cpu().numpy(), H, w.head_dim)
+        rep["qkv_projection"] = stage([host(t[k_][rows]) for k_ in ("q", "k", "v")], list(want))
+    got, ref = [], []
+    for f in frames:
+        sl = slice(f * T, (f + 1) * T)
+        Q, K, V = (host(t[k_][sl]) for k_ in ("q", "k", "v"))
+        rows, heads = g.integers(0, T, 64), g.integers(0, H, 64)
+        ref.append(layer_io.frame_attention_rows(Q, K, V, T, rows, heads))
+        o = t["o"][sl]
+        got.append(host(o[torch.as_tensor(rows, device=dev), torch.as_tensor(heads, device=dev)]))
+    rep["frame_attention"] = stage(got, ref)
+    if "y" in t:
+        rows = torch.as_tensor([f * T + int(r) for f in frames for r in g.integers(0, T, 16)], device=dev)
+        want = layer_io.out_project(host(t["o"][rows]), host(t["w_o"]), t["b_o"].cpu().numpy())
+        rep["out_projection"] = stage([host(t["y"][rows])], [want])
+    return rep
+
+
 def bench_block(args, w, world, rank, local, dist):
     """One step = the frame-wise attention layer, or a whole block (QKV projection, attention,
     output projection), on synthetic tokens and random-init weights resident in HBM."""
@@ -651,6 +689,8 @@ def bench_block(args, w, world, rank, local, dist):
         ms, threads, host_cpus, sample = oracle_block_sample(w, budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": ms, "unit": UNIT, "cores": threads, "host_cpus": host_cpus,
                                 "kind": "oracle", "extrapolated": True, "sample": sample}
+        if w.kind in ("frame", "frame_block"):
+            line["parity_sample"] = block_parity_sample(torch, w, t)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist:
