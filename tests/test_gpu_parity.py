@@ -154,6 +154,26 @@ def test_long500_mask_full_and_sampled_rows():
         assert rel_l2(got, ref) <= BF16_TOL[0] and max_abs(got, ref) <= BF16_TOL[1]
 
 
+@pytest.mark.slow
+def test_long_rows_twelve_row_mask_variant():
+    """B = 3,643 blocks (600 frames, 2 heads): past the 14-row long-row CTA's shared memory, so
+    the mask kernel runs 12 rows per CTA; every row against the oracle."""
+    import torch
+    from view_transformers_b200 import layer
+    w = configs.LONG500.with_(name="long600_h2", frames=600, heads=2, tau=0.0)
+    x = inputs(w)
+    L = layer.BlockSparseLayer.for_workload(w)
+    assert L.B == 3643
+    q, k = (layer.to_device(a, w.dtype) for a in (x.q, x.k))
+    L.predict(q, k)
+    torch.cuda.synchronize()
+    assert L.check_status() == 0
+    lay, PQ, PK, kh, om = _oracle_mask(w, x, {})
+    rep = compare_mask(om, L.selected(), w.tau)
+    print(f"long600_h2: mask rows {rep.rows} exact {rep.exact} exempt {rep.exempt} failed {rep.failed}")
+    assert rep.ok, rep.failures
+
+
 # ------------------------------------------------------------------ edge cases
 
 EDGE = [
